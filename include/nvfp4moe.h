@@ -1,0 +1,269 @@
+/*
+ * nvfp4moe -- NVFP4 W4A4 MoE expert layer for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the MoE expert linear layer of miniTE's NVFP4 learner:
+ *   news.hamidun.com "miniTE ... 1.39x over BF16 on Qwen3-30B-A3B" (Arabic and
+ *   Russian editions), key facts: native NVFP4 W4A4 (4-bit weights and
+ *   activations); section "diagnostics, alignment and fast kernels": grouped
+ *   GEMMs over the many experts of Qwen3-30B-A3B; strict-alignment mode.
+ *   www.aib.vote "miniTE report, NVFP4 RL stability", paragraph 4: the
+ *   token-wise NVFP4 path of Transformer Engine -- contiguous data layout,
+ *   device-side metadata, amax reuse, grouped matrix multiplication and
+ *   operator fusion.
+ *
+ * Data formats (the pages name NVFP4; the format itself is the public NVFP4
+ * definition):
+ *   codes   E2M1, two per byte, element 2i in the low nibble of byte i
+ *   scales  one UE4M3 byte per 16 consecutive elements along K
+ *   S_dec   FP32 decode scale, per tensor or per row; x ~ e2m1 * sf * S_dec
+ *   Quantization: amax -> S_enc = 2688/amax, S_dec = 1/S_enc (binary32);
+ *   sf = UE4M3_rne_satfinite((bamax/6)*S_enc); code = E2M1_rne_satfinite(x*S_enc/sf).
+ *
+ * Scale-factor layouts
+ *   row-major     scales[row][K/16]
+ *   MMA layout    the 128-row x 4-scale atom the tcgen05 block-scaled MMA reads:
+ *                 byte(row, b) = ((row/128)*(K/64) + b/4)*512 + (row%32)*16
+ *                                + ((row%128)/32)*4 + b%4
+ *                 (rows of a matrix padded to a multiple of 128).
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless the comment says host.  The caller
+ *     owns and allocates every buffer (workspace included); the library never
+ *     allocates device memory and never synchronizes the host, except
+ *     nvfp4moe_device_status() which says so.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is stream-ordered.
+ *   - Argument, shape and alignment errors are returned before anything is
+ *     launched.  A CUDA launch error is returned as NVFP4MOE_ERR_CUDA.  Errors
+ *     the kernels detect (an expert index out of range, a duplicate expert in
+ *     one token's top-k, a wait that timed out) are recorded in an error word
+ *     inside the caller's workspace and read with nvfp4moe_device_status().
+ *   - Device pointers must be 16-byte aligned; sizes: K % 256 == 0 and
+ *     N % 256 == 0 for the grouped GEMM, K % 64 == 0 for the quantizer.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *nvfp4moe_stream_t;
+
+typedef enum {
+  NVFP4MOE_OK = 0,
+  NVFP4MOE_ERR_INVALID_ARG = -1,      /* null pointer, negative size, bad flag   */
+  NVFP4MOE_ERR_MISALIGNED = -2,       /* a pointer is not 16-byte aligned        */
+  NVFP4MOE_ERR_UNSUPPORTED_SHAPE = -3,/* K, N or E outside what the kernels take */
+  NVFP4MOE_ERR_CUDA = -4,             /* a CUDA runtime / driver call failed     */
+  NVFP4MOE_ERR_DEVICE_TIMEOUT = -5,   /* a kernel wait ran out (device status)   */
+  NVFP4MOE_ERR_WORKSPACE = -6,        /* workspace missing or too small          */
+  NVFP4MOE_ERR_DEVICE_CHECK = -7      /* kernel-side input check failed (device status) */
+} nvfp4moe_status;
+
+/* ---------------------------------------------------------------- flags -- */
+/* One FP32 global scale per row (token) instead of one per tensor. */
+#define NVFP4MOE_SCALE_PER_TOKEN 0x1u
+/* Strict alignment (the pages' strict-alignment mode): per-token scales and a
+ * reduction order fixed per output element, so each token's output is bitwise
+ * identical however the tokens are batched, ordered or grouped. */
+#define NVFP4MOE_STRICT 0x2u
+/* Scale factors are written / read in the MMA atom layout (see above). */
+#define NVFP4MOE_SF_MMA_LAYOUT 0x4u
+/* Grouped GEMM: write output rows at their padded positions instead of the
+ * compact sorted positions. */
+#define NVFP4MOE_OUT_PADDED 0x8u
+/* nvfp4_prepare_weights: the matrix is a fused gate_up [2I][K] (gate rows
+ * 0..I-1, up rows I..2I-1); store rows in the order the fused SwiGLU epilogue
+ * reads (per 256-row tile: 128 gate rows then the matching 128 up rows). */
+#define NVFP4MOE_W_GATE_UP 0x10u
+
+const char *nvfp4moe_status_string(int status);
+int nvfp4moe_version(void);
+
+/* Reads and clears the error word of a workspace (the first 16 bytes of every
+ * workspace this library uses): synchronizes `stream`, copies the word to the
+ * host, zeroes it, and returns NVFP4MOE_OK, NVFP4MOE_ERR_DEVICE_CHECK or
+ * NVFP4MOE_ERR_DEVICE_TIMEOUT.  This is the one call that blocks the host. */
+int nvfp4moe_device_status(void *workspace, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------ quantize -- */
+/* NVFP4-quantize x [M][K] BF16 (row-major).  The token-wise NVFP4 path with
+ * amax reuse (www.aib.vote "miniTE report", paragraph 4).
+ *   amax_in   nullable.  Per-tensor mode: [1]; per-token: [M].  When given,
+ *             it is used as is (amax reuse) and no amax pass runs.
+ *   amax_out  nullable, same shape; receives the amax used.  In per-tensor
+ *             mode without amax_in it is REQUIRED (the reduction target).
+ *   q         [M][K/2] packed E2M1 codes (out)
+ *   scales    UE4M3 scales, row-major [M][K/16] or, with
+ *             NVFP4MOE_SF_MMA_LAYOUT, the MMA layout over roundup(M,128) rows
+ *   s_dec     [1] (per tensor) or [M] (per token) FP32 decode scales (out)
+ *   flags     NVFP4MOE_SCALE_PER_TOKEN | NVFP4MOE_STRICT | NVFP4MOE_SF_MMA_LAYOUT
+ * Requirements: K % 64 == 0, M >= 0 (M == 0 is a no-op). */
+int nvfp4_quantize(const void *x, int64_t M, int64_t K, const float *amax_in,
+                   float *amax_out, uint8_t *q, uint8_t *scales, float *s_dec,
+                   uint32_t flags, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------- permute -- */
+/* Token-to-expert permutation into a contiguous per-expert layout with
+ * device-side group offsets (www.aib.vote "miniTE report", paragraph 4:
+ * contiguous layout, device-side metadata).  Rows are ordered by
+ * (expert, token, slot); the host never learns the group sizes.
+ *   topk_idx        [T][k] int32 expert ids; each row holds k distinct ids
+ *   offsets         [E+1] int32 (out): group e is rows offsets[e]..offsets[e+1]
+ *   padded_offsets  [E+1] int32 (out): the same with every group rounded up
+ *                   to a multiple of 128 rows (the GEMM tile height)
+ *   perm            [T*k] int32 (out): perm[r] = t*k + j for sorted row r
+ *   inv_perm        [T][k] int32 (out): inv_perm[t][j] = r
+ *   workspace       moe_permute_workspace_size() bytes
+ * Out-of-range or duplicate expert ids set NVFP4MOE_ERR_DEVICE_CHECK in the
+ * workspace error word; such entries are skipped, nothing is written out of
+ * bounds.  Requirements: 1 <= E <= 1024, 1 <= k <= 32. */
+size_t moe_permute_workspace_size(int64_t T, int k, int E);
+int moe_permute(const int32_t *topk_idx, int64_t T, int k, int E,
+                int32_t *offsets, int32_t *padded_offsets, int32_t *perm,
+                int32_t *inv_perm, void *workspace, size_t workspace_bytes,
+                nvfp4moe_stream_t stream);
+
+/* Quantize each token of x [T][K] once and write its codes, scales and
+ * decode scale to all k of its rows in the padded grouped layout (the fused
+ * quantize + permute of the token-wise path: amax computed once, reused for
+ * every copy).  Uses the inv_perm / offsets / padded_offsets of moe_permute.
+ *   q_rows      [rows_cap][K/2] codes at padded row positions (out)
+ *   sf_rows     MMA-layout scales over rows_cap rows (out)
+ *   s_dec_rows  [rows_cap] FP32 per-row decode scale (out; per-tensor mode
+ *               writes the tensor's S_dec into every row)
+ *   amax_in / amax_out as for nvfp4_quantize (per tensor [1], per token [T])
+ *   rows_cap    allocated padded rows: >= roundup(T*k + E*127, 128)
+ * flags: NVFP4MOE_SCALE_PER_TOKEN | NVFP4MOE_STRICT. */
+int moe_quantize_permute(const void *x, int64_t T, int64_t K, int k, int E,
+                         const int32_t *topk_idx, const int32_t *inv_perm,
+                         const int32_t *offsets, const int32_t *padded_offsets,
+                         const float *amax_in, float *amax_out, uint8_t *q_rows,
+                         uint8_t *sf_rows, float *s_dec_rows, int64_t rows_cap,
+                         uint32_t flags, nvfp4moe_stream_t stream);
+
+/* --------------------------------------------------------- grouped GEMM -- */
+/* Block-scaled FP4 x FP4 grouped GEMM over the experts, one launch, group
+ * sizes read on the device (news.hamidun.com section "diagnostics, alignment
+ * and fast kernels": grouped GEMMs for MoE; www.aib.vote paragraph 4).
+ * For every expert e and every row r of its group:
+ *   out[r][n] = S_dec_a(r) * S_dec_w[e] * sum_k a(r,k) * w(e,n,k)
+ * with a, w the block-scaled E2M1 values; FP32 accumulation in the tensor
+ * cores, one rounding to the output type.
+ *   q_a, sf_a, s_dec_a  A in the padded grouped layout (moe_quantize_permute):
+ *                       q_a [rows_cap][K/2], sf_a MMA layout, s_dec_a
+ *                       [rows_cap] (NVFP4MOE_SCALE_PER_TOKEN) or [1]
+ *   q_w, sf_w, s_dec_w  weights: q_w [E][N][K/2], sf_w MMA layout per expert
+ *                       ([E][N/128][K/64][512] bytes), s_dec_w [E]
+ *   offsets, padded_offsets  [E+1] device group offsets (moe_permute)
+ *   out_bf16, out_f32   nullable (at least one): [R][N] compact sorted rows,
+ *                       or [rows_cap][N] with NVFP4MOE_OUT_PADDED
+ *   workspace           16 bytes at least (error word)
+ * Requirements: K % 256 == 0, N % 256 == 0, 1 <= E. */
+int nvfp4_grouped_gemm(const uint8_t *q_a, const uint8_t *sf_a,
+                       const float *s_dec_a, const uint8_t *q_w,
+                       const uint8_t *sf_w, const float *s_dec_w,
+                       const int32_t *offsets, const int32_t *padded_offsets,
+                       int E, int64_t rows_cap, int64_t N, int64_t K,
+                       void *out_bf16, float *out_f32, uint32_t flags,
+                       void *workspace, size_t workspace_bytes,
+                       nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------- weights -- */
+/* NVFP4 weights of one MoE linear, E experts of [N][K] each, every expert
+ * one tensor (one S_dec per expert).  All pointers are device pointers. */
+typedef struct {
+  uint8_t *q;      /* [E][N][K/2] packed codes, rows in kernel order        */
+  uint8_t *sf;     /* [E][N/128][K/64][512] UE4M3, MMA layout              */
+  float *s_dec;    /* [E] decode scales                                     */
+  float *amax;     /* [E] amax of each expert's BF16 matrix                 */
+  int64_t E, N, K;
+  uint32_t flags;  /* NVFP4MOE_W_GATE_UP when rows are gate/up interleaved  */
+} nvfp4moe_weights;
+
+/* Quantize BF16 weights w [E][N][K] into `out` (whose q/sf/s_dec/amax buffers
+ * the caller allocated).  One-time preparation, not part of the layer step.
+ * flags: NVFP4MOE_W_GATE_UP to store the fused gate_up rows interleaved.
+ * Requirements: K % 256 == 0, N % 256 == 0 (gate_up: N/2 % 128 == 0). */
+int nvfp4_prepare_weights(const void *w, int64_t E, int64_t N, int64_t K,
+                          uint32_t flags, nvfp4moe_weights *out,
+                          nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------- combine -- */
+/* y[t] = BF16( sum_{j<k} topk_w[t][j] * D[inv_perm[t][j]] ), FP32 sum in slot
+ * order j = 0..k-1 (a fixed order: the strict-alignment requirement).
+ *   d        [R][H] BF16 expert outputs in compact sorted order
+ *   inv_perm [T][k], topk_w [T][k] FP32, y [T][H] BF16 (out)
+ * Requirements: H % 8 == 0. */
+int moe_combine(const void *d, const int32_t *inv_perm, const float *topk_w,
+                int64_t T, int k, int64_t H, void *y, nvfp4moe_stream_t stream);
+
+/* --------------------------------------------------------- the layer ---- */
+/* The whole W4A4 MoE expert layer, one stream, no host synchronization:
+ *   quantize x once per token + permute (fused)  -> gate_up grouped GEMM with
+ *   a fused SwiGLU epilogue that also reduces the amax of h  -> requantize h
+ *   reusing that amax  -> down grouped GEMM  -> weighted combine.
+ *   x         [T][H] BF16 activations
+ *   topk_idx  [T][k] int32, topk_w [T][k] FP32 routing (router output)
+ *   w_gate_up prepared with NVFP4MOE_W_GATE_UP: E x [2I][H]
+ *   w_down    prepared plainly: E x [H][I]
+ *   y         [T][H] BF16 (out)
+ *   flags     NVFP4MOE_SCALE_PER_TOKEN | NVFP4MOE_STRICT
+ *   workspace moe_expert_layer_workspace_size() bytes; its named regions
+ *             (offsets, perm, h, ...) are laid out by
+ *             moe_expert_layer_workspace_offsets() for inspection.
+ * Requirements: H % 256 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32. */
+size_t moe_expert_layer_workspace_size(int64_t T, int64_t H, int64_t I, int E,
+                                       int k, uint32_t flags);
+
+/* Byte offsets of the regions inside the layer workspace, in this order:
+ * [0] error word, [1] offsets, [2] padded_offsets, [3] perm, [4] inv_perm,
+ * [5] x codes (padded rows), [6] x scales (MMA layout), [7] x row S_dec,
+ * [8] h BF16 (padded rows), [9] h amax, [10] h codes, [11] h scales,
+ * [12] h row S_dec, [13] D BF16 (compact rows), [14] rows_cap (a count, not an
+ * offset), [15] total bytes.  `out` must hold 16 int64 (host memory). */
+int moe_expert_layer_workspace_offsets(int64_t T, int64_t H, int64_t I, int E,
+                                       int k, uint32_t flags, int64_t *out);
+
+int moe_expert_layer(const void *x, const int32_t *topk_idx,
+                     const float *topk_w, const nvfp4moe_weights *w_gate_up,
+                     const nvfp4moe_weights *w_down, int64_t T, int64_t H,
+                     int64_t I, int E, int k, void *y, uint32_t flags,
+                     void *workspace, size_t workspace_bytes,
+                     nvfp4moe_stream_t stream);
+
+/* moe_expert_layer that also records CUDA events at its stage boundaries, so
+ * a caller can time each kernel on the stream it runs on.  stage_events
+ * (host array of 7 cudaEvent_t, entries may be NULL): [0] before the first
+ * launch, [1] after routing (counts, amax, offsets), [2] after the fused
+ * quantize + permute, [3] after the gate_up GEMM + SwiGLU, [4] after the
+ * requantization of h, [5] after the down GEMM, [6] after the combine.
+ * Everything else is exactly moe_expert_layer. */
+int moe_expert_layer_profiled(const void *x, const int32_t *topk_idx,
+                              const float *topk_w,
+                              const nvfp4moe_weights *w_gate_up,
+                              const nvfp4moe_weights *w_down, int64_t T,
+                              int64_t H, int64_t I, int E, int k, void *y,
+                              uint32_t flags, void *workspace,
+                              size_t workspace_bytes, nvfp4moe_stream_t stream,
+                              void *const *stage_events);
+
+/* ---------------------------------------------------------- diagnostics -- */
+/* The hardware conversions the quantizer uses, exposed so their rounding can
+ * be checked against the format definition: codes[i] = E2M1_rne_satfinite(y[i])
+ * (one code per byte, 0..15) and codes[i] = UE4M3_rne_satfinite(v[i]). */
+int nvfp4moe_encode_e2m1(const float *y, int64_t n, uint8_t *codes,
+                         nvfp4moe_stream_t stream);
+int nvfp4moe_encode_ue4m3(const float *v, int64_t n, uint8_t *codes,
+                          nvfp4moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4MOE_H */

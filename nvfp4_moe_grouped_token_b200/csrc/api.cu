@@ -1,0 +1,576 @@
+// The C-ABI of nvfp4moe: argument checks, workspace layout and the layer's
+// launch sequence.  Plain pointers and sizes only; see include/nvfp4moe.h.
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4moe {
+
+int num_sms() {
+  static int cache[64];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (int i = 0; i < 64; ++i) cache[i] = 0;
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace nvfp4moe
+
+using namespace nvfp4moe;
+
+namespace {
+
+constexpr int64_t kAlign = 256;
+constexpr int64_t kHeaderBytes = 256;     // error word, detail, x amax, h amax
+constexpr int64_t kHdrXAmax = 16;         // byte offsets inside the header
+constexpr int64_t kHdrHAmax = 20;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA; }
+cudaStream_t st(nvfp4moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+#define NVFP4MOE_TRY(expr)                 \
+  do {                                     \
+    cudaError_t e_ = (expr);               \
+    if (e_ != cudaSuccess) return NVFP4MOE_ERR_CUDA; \
+  } while (0)
+
+// Bump allocator over a caller-provided workspace.
+struct Carve {
+  int64_t off = 0;
+  int64_t take(int64_t bytes) {
+    const int64_t o = off;
+    off += round_up(bytes > 0 ? bytes : 0, kAlign);
+    return o;
+  }
+};
+
+struct PermuteLayout {
+  int64_t hdr, counts, local_rank, total;
+};
+
+PermuteLayout permute_layout(int64_t T, int k, int E) {
+  Carve c;
+  PermuteLayout L;
+  L.hdr = c.take(kHeaderBytes);
+  L.counts = c.take(permute_blocks(T) * E * 4);
+  L.local_rank = c.take(T * k * 4);
+  L.total = c.off;
+  return L;
+}
+
+int64_t layer_rows_cap(int64_t T, int k, int E) { return round_up(T * k + 127 * (int64_t)E, 128); }
+
+struct LayerLayout {
+  int64_t v[16];
+  int64_t counts, local_rank;
+};
+
+LayerLayout layer_layout(int64_t T, int64_t H, int64_t I, int E, int k) {
+  const int64_t R = T * k;
+  const int64_t cap = layer_rows_cap(T, k, E);
+  Carve c;
+  LayerLayout L;
+  L.v[0] = c.take(kHeaderBytes);
+  L.v[1] = c.take((E + 1) * 4);
+  L.v[2] = c.take((E + 1) * 4);
+  L.v[3] = c.take(R * 4);
+  L.v[4] = c.take(R * 4);
+  L.v[5] = c.take(cap * H / 2);
+  L.v[6] = c.take(cap * H / 16);
+  L.v[7] = c.take(cap * 4);
+  L.v[8] = c.take(cap * I * 2);
+  L.v[9] = c.take(cap * 4);
+  L.v[10] = c.take(cap * I / 2);
+  L.v[11] = c.take(cap * I / 16);
+  L.v[12] = c.take(cap * 4);
+  L.v[13] = c.take(R * H * 2);
+  L.counts = c.take(permute_blocks(T) * E * 4);
+  L.local_rank = c.take(R * 4);
+  L.v[14] = cap;
+  L.v[15] = c.off;
+  return L;
+}
+
+bool per_token(uint32_t flags) { return (flags & (NVFP4MOE_SCALE_PER_TOKEN | NVFP4MOE_STRICT)) != 0; }
+
+int check_weights(const nvfp4moe_weights *w, int64_t E, int64_t N, int64_t K) {
+  if (w == nullptr || w->q == nullptr || w->sf == nullptr || w->s_dec == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (w->E != E || w->N != N || w->K != K) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(w->q) || !aligned16(w->sf)) return NVFP4MOE_ERR_MISALIGNED;
+  return NVFP4MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *nvfp4moe_status_string(int status) {
+  switch (status) {
+    case NVFP4MOE_OK: return "ok";
+    case NVFP4MOE_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4MOE_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case NVFP4MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4MOE_ERR_CUDA: return "CUDA error";
+    case NVFP4MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case NVFP4MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4MOE_ERR_DEVICE_CHECK: return "device-side input check failed";
+    default: return "unknown status";
+  }
+}
+
+int nvfp4moe_version(void) { return 100; }
+
+int nvfp4moe_device_status(void *workspace, nvfp4moe_stream_t stream) {
+  if (workspace == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  int words[2] = {0, 0};
+  NVFP4MOE_TRY(cudaStreamSynchronize(st(stream)));
+  NVFP4MOE_TRY(cudaMemcpy(words, workspace, sizeof(words), cudaMemcpyDeviceToHost));
+  NVFP4MOE_TRY(cudaMemset(workspace, 0, sizeof(words)));
+  if (words[0] == kDevOk) return NVFP4MOE_OK;
+  if (words[0] == kDevTimeout) return NVFP4MOE_ERR_DEVICE_TIMEOUT;
+  return NVFP4MOE_ERR_DEVICE_CHECK;
+}
+
+int nvfp4_quantize(const void *x, int64_t M, int64_t K, const float *amax_in, float *amax_out,
+                   uint8_t *q, uint8_t *scales, float *s_dec, uint32_t flags,
+                   nvfp4moe_stream_t stream) {
+  if (M < 0 || K <= 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (K % 64 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return NVFP4MOE_OK;
+  if (x == nullptr || q == nullptr || scales == nullptr || s_dec == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(scales)) return NVFP4MOE_ERR_MISALIGNED;
+  const bool tok = per_token(flags);
+  if (!tok && amax_in == nullptr && amax_out == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  cudaStream_t s = st(stream);
+  QuantParams p;
+  p.x = x;
+  p.tasks = M;
+  p.K = K;
+  p.mode = kQuantPlain;
+  p.q = q;
+  p.sf = scales;
+  p.sf_mma = (flags & NVFP4MOE_SF_MMA_LAYOUT) ? 1 : 0;
+  p.s_dec = s_dec;
+  p.s_dec_rows = tok ? 1 : 0;
+  p.rows_cap = M;
+  if (tok) {
+    p.amax_rows = 1;
+    if (amax_in != nullptr) {
+      p.amax_src = amax_in;
+      if (amax_out != nullptr && amax_out != amax_in)
+        NVFP4MOE_TRY(cudaMemcpyAsync(amax_out, amax_in, M * 4, cudaMemcpyDeviceToDevice, s));
+    } else {
+      p.compute_row_amax = 1;
+      p.amax_out = amax_out;
+    }
+  } else {
+    if (amax_in != nullptr) {
+      p.amax_src = amax_in;
+      if (amax_out != nullptr && amax_out != amax_in)
+        NVFP4MOE_TRY(cudaMemcpyAsync(amax_out, amax_in, 4, cudaMemcpyDeviceToDevice, s));
+    } else {
+      NVFP4MOE_TRY(cudaMemsetAsync(amax_out, 0, 4, s));
+      NVFP4MOE_TRY(launch_amax(x, M * K, 1, amax_out, s));
+      p.amax_src = amax_out;
+    }
+  }
+  return cuda_rc(launch_quant(p, s));
+}
+
+size_t moe_permute_workspace_size(int64_t T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  return (size_t)permute_layout(T, k, E).total;
+}
+
+int moe_permute(const int32_t *topk_idx, int64_t T, int k, int E, int32_t *offsets,
+                int32_t *padded_offsets, int32_t *perm, int32_t *inv_perm, void *workspace,
+                size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > 32 || E < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (offsets == nullptr || padded_offsets == nullptr || (T > 0 && (topk_idx == nullptr || perm == nullptr || inv_perm == nullptr)))
+    return NVFP4MOE_ERR_INVALID_ARG;
+  const PermuteLayout L = permute_layout(T, k, E);
+  if (workspace == nullptr || (int64_t)workspace_bytes < L.total) return NVFP4MOE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  NVFP4MOE_TRY(cudaMemsetAsync(ws + L.hdr, 0, 16, s));
+  PermuteParams p;
+  p.topk_idx = topk_idx;
+  p.T = T;
+  p.k = k;
+  p.E = E;
+  p.block_counts = reinterpret_cast<int32_t *>(ws + L.counts);
+  p.local_rank = reinterpret_cast<int32_t *>(ws + L.local_rank);
+  p.offsets = offsets;
+  p.padded_offsets = padded_offsets;
+  p.perm = perm;
+  p.inv_perm = inv_perm;
+  p.err = reinterpret_cast<int *>(ws + L.hdr);
+  NVFP4MOE_TRY(launch_route_count(p, s));
+  NVFP4MOE_TRY(launch_route_scan(p, s));
+  NVFP4MOE_TRY(launch_route_rank(p, s));
+  return NVFP4MOE_OK;
+}
+
+int moe_quantize_permute(const void *x, int64_t T, int64_t K, int k, int E, const int32_t *topk_idx,
+                         const int32_t *inv_perm, const int32_t *offsets,
+                         const int32_t *padded_offsets, const float *amax_in, float *amax_out,
+                         uint8_t *q_rows, uint8_t *sf_rows, float *s_dec_rows, int64_t rows_cap,
+                         uint32_t flags, nvfp4moe_stream_t stream) {
+  if (T < 0 || K <= 0 || k < 1 || k > 32 || E < 1 || rows_cap < 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (K % 64 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return NVFP4MOE_OK;
+  if (x == nullptr || topk_idx == nullptr || inv_perm == nullptr || offsets == nullptr ||
+      padded_offsets == nullptr || q_rows == nullptr || sf_rows == nullptr || s_dec_rows == nullptr)
+    return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q_rows) || !aligned16(sf_rows)) return NVFP4MOE_ERR_MISALIGNED;
+  const bool tok = per_token(flags);
+  if (!tok && amax_in == nullptr && amax_out == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  cudaStream_t s = st(stream);
+  QuantParams p;
+  p.x = x;
+  p.tasks = T;
+  p.K = K;
+  p.mode = kQuantScatter;
+  p.q = q_rows;
+  p.sf = sf_rows;
+  p.sf_mma = 1;
+  p.s_dec = s_dec_rows;
+  p.s_dec_rows = 1;
+  p.rows_cap = rows_cap;
+  p.topk_idx = topk_idx;
+  p.inv_perm = inv_perm;
+  p.offsets = offsets;
+  p.padded_offsets = padded_offsets;
+  p.k = k;
+  p.E = E;
+  if (tok) {
+    p.amax_rows = 1;
+    if (amax_in != nullptr) {
+      p.amax_src = amax_in;
+    } else {
+      p.compute_row_amax = 1;
+      p.amax_out = amax_out;
+    }
+  } else {
+    if (amax_in != nullptr) {
+      p.amax_src = amax_in;
+    } else {
+      NVFP4MOE_TRY(cudaMemsetAsync(amax_out, 0, 4, s));
+      NVFP4MOE_TRY(launch_amax(x, T * K, 1, amax_out, s));
+      p.amax_src = amax_out;
+    }
+  }
+  return cuda_rc(launch_quant(p, s));
+}
+
+int nvfp4_grouped_gemm(const uint8_t *q_a, const uint8_t *sf_a, const float *s_dec_a,
+                       const uint8_t *q_w, const uint8_t *sf_w, const float *s_dec_w,
+                       const int32_t *offsets, const int32_t *padded_offsets, int E, int64_t rows_cap,
+                       int64_t N, int64_t K, void *out_bf16, float *out_f32, uint32_t flags,
+                       void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (E < 1 || rows_cap < 0 || N <= 0 || K <= 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (K % 256 != 0 || N % 256 != 0 || rows_cap % 128 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (q_a == nullptr || sf_a == nullptr || s_dec_a == nullptr || q_w == nullptr || sf_w == nullptr ||
+      s_dec_w == nullptr || offsets == nullptr || padded_offsets == nullptr ||
+      (out_bf16 == nullptr && out_f32 == nullptr))
+    return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(q_a) || !aligned16(sf_a) || !aligned16(q_w) || !aligned16(sf_w) ||
+      !aligned16(out_bf16) || !aligned16(out_f32))
+    return NVFP4MOE_ERR_MISALIGNED;
+  if (workspace == nullptr || workspace_bytes < 16) return NVFP4MOE_ERR_WORKSPACE;
+  if (rows_cap == 0) return NVFP4MOE_OK;
+  cudaStream_t s = st(stream);
+  NVFP4MOE_TRY(cudaMemsetAsync(workspace, 0, 16, s));
+  GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q_a = q_a;
+  a.sf_a = sf_a;
+  a.s_dec_a = s_dec_a;
+  a.s_dec_a_rows = per_token(flags) ? 1 : 0;
+  a.q_w = q_w;
+  a.sf_w = sf_w;
+  a.s_dec_w = s_dec_w;
+  a.offsets = offsets;
+  a.padded_offsets = padded_offsets;
+  a.E = E;
+  a.rows_cap = rows_cap;
+  a.N = N;
+  a.K = K;
+  a.epilogue = kEpiStore;
+  a.out_bf16 = out_bf16;
+  a.out_f32 = out_f32;
+  a.out_padded = (flags & NVFP4MOE_OUT_PADDED) ? 1 : 0;
+  a.err = static_cast<int *>(workspace);
+  return cuda_rc(launch_grouped_gemm(a, s));
+}
+
+int nvfp4_prepare_weights(const void *w, int64_t E, int64_t N, int64_t K, uint32_t flags,
+                          nvfp4moe_weights *out, nvfp4moe_stream_t stream) {
+  if (w == nullptr || out == nullptr || E < 1 || N <= 0 || K <= 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (out->q == nullptr || out->sf == nullptr || out->s_dec == nullptr || out->amax == nullptr)
+    return NVFP4MOE_ERR_INVALID_ARG;
+  if (K % 256 != 0 || N % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  const bool gate_up = (flags & NVFP4MOE_W_GATE_UP) != 0;
+  if (gate_up && (N / 2) % 128 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(w) || !aligned16(out->q) || !aligned16(out->sf)) return NVFP4MOE_ERR_MISALIGNED;
+  cudaStream_t s = st(stream);
+  NVFP4MOE_TRY(cudaMemsetAsync(out->amax, 0, E * 4, s));
+  NVFP4MOE_TRY(launch_amax(w, N * K, E, out->amax, s));
+  QuantParams p;
+  p.x = w;
+  p.tasks = E * N;
+  p.K = K;
+  p.mode = kQuantWeights;
+  p.amax_src = out->amax;
+  p.amax_rows = 1;
+  p.q = out->q;
+  p.sf = out->sf;
+  p.sf_mma = 1;
+  p.s_dec = out->s_dec;
+  p.s_dec_rows = 0;
+  p.rows_cap = E * N;
+  p.N = N;
+  p.gate_up = gate_up ? 1 : 0;
+  NVFP4MOE_TRY(launch_quant(p, s));
+  out->E = E;
+  out->N = N;
+  out->K = K;
+  out->flags = gate_up ? NVFP4MOE_W_GATE_UP : 0u;
+  return NVFP4MOE_OK;
+}
+
+int moe_combine(const void *d, const int32_t *inv_perm, const float *topk_w, int64_t T, int k,
+                int64_t H, void *y, nvfp4moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > 32 || H <= 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return NVFP4MOE_OK;
+  if (d == nullptr || inv_perm == nullptr || topk_w == nullptr || y == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(d) || !aligned16(y)) return NVFP4MOE_ERR_MISALIGNED;
+  return cuda_rc(launch_combine(d, inv_perm, topk_w, T, k, H, y, st(stream)));
+}
+
+size_t moe_expert_layer_workspace_size(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
+  (void)flags;
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+  return (size_t)layer_layout(T, H, I, E, k).v[15];
+}
+
+int moe_expert_layer_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags,
+                                       int64_t *out) {
+  (void)flags;
+  if (out == nullptr || T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  const LayerLayout L = layer_layout(T, H, I, E, k);
+  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
+  return NVFP4MOE_OK;
+}
+
+static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float *topk_w,
+                             const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down,
+                             int64_t T, int64_t H, int64_t I, int E, int k, void *y, uint32_t flags,
+                             void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream,
+                             void *const *events) {
+  if (T < 0 || H <= 0 || I <= 0 || k < 1 || k > 32 || E < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || H % 256 != 0 || I % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_weights(w_gate_up, E, 2 * I, H);
+  if (rc != NVFP4MOE_OK) return rc;
+  if (!(w_gate_up->flags & NVFP4MOE_W_GATE_UP)) return NVFP4MOE_ERR_INVALID_ARG;
+  rc = check_weights(w_down, E, H, I);
+  if (rc != NVFP4MOE_OK) return rc;
+  if (T == 0) return NVFP4MOE_OK;
+  if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || y == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  const LayerLayout L = layer_layout(T, H, I, E, k);
+  if (workspace == nullptr || (int64_t)workspace_bytes < L.v[15]) return NVFP4MOE_ERR_WORKSPACE;
+  const bool tok = per_token(flags);
+  const int64_t cap = L.v[14];
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int *err = reinterpret_cast<int *>(ws + L.v[0]);
+  float *x_amax = reinterpret_cast<float *>(ws + L.v[0] + kHdrXAmax);
+  float *h_amax_tensor = reinterpret_cast<float *>(ws + L.v[0] + kHdrHAmax);
+  int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.v[1]);
+  int32_t *padded = reinterpret_cast<int32_t *>(ws + L.v[2]);
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.v[3]);
+  int32_t *inv_perm = reinterpret_cast<int32_t *>(ws + L.v[4]);
+  uint8_t *xq = ws + L.v[5];
+  uint8_t *xsf = ws + L.v[6];
+  float *xsd = reinterpret_cast<float *>(ws + L.v[7]);
+  void *hb = ws + L.v[8];
+  float *h_amax_rows = reinterpret_cast<float *>(ws + L.v[9]);
+  uint8_t *hq = ws + L.v[10];
+  uint8_t *hsf = ws + L.v[11];
+  float *hsd = reinterpret_cast<float *>(ws + L.v[12]);
+  void *d = ws + L.v[13];
+
+  auto mark = [&](int i) -> cudaError_t {
+    if (events == nullptr || events[i] == nullptr) return cudaSuccess;
+    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]), s);
+  };
+  NVFP4MOE_TRY(mark(0));
+  NVFP4MOE_TRY(cudaMemsetAsync(ws + L.v[0], 0, kHeaderBytes, s));
+
+  // 1-2. route counts, (per-tensor) amax of x, offsets
+  PermuteParams pp;
+  pp.topk_idx = topk_idx;
+  pp.T = T;
+  pp.k = k;
+  pp.E = E;
+  pp.block_counts = reinterpret_cast<int32_t *>(ws + L.counts);
+  pp.local_rank = reinterpret_cast<int32_t *>(ws + L.local_rank);
+  pp.offsets = offsets;
+  pp.padded_offsets = padded;
+  pp.perm = perm;
+  pp.inv_perm = inv_perm;
+  pp.err = err;
+  NVFP4MOE_TRY(launch_route_count(pp, s));
+  if (!tok) NVFP4MOE_TRY(launch_amax(x, T * H, 1, x_amax, s));
+  NVFP4MOE_TRY(launch_route_scan(pp, s));
+  NVFP4MOE_TRY(mark(1));
+
+  // 3. quantize each token once, scatter to its k rows, write perm / inv_perm
+  QuantParams q;
+  q.x = x;
+  q.tasks = T;
+  q.K = H;
+  q.mode = kQuantScatter;
+  q.q = xq;
+  q.sf = xsf;
+  q.sf_mma = 1;
+  q.s_dec = xsd;
+  q.s_dec_rows = 1;
+  q.rows_cap = cap;
+  q.topk_idx = topk_idx;
+  q.offsets = offsets;
+  q.padded_offsets = padded;
+  q.k = k;
+  q.E = E;
+  q.local_rank = pp.local_rank;
+  q.block_base = pp.block_counts;
+  q.perm_out = perm;
+  q.inv_perm_out = inv_perm;
+  q.zero_rows = tok ? h_amax_rows : nullptr;
+  if (tok) {
+    q.amax_rows = 1;
+    q.compute_row_amax = 1;
+  } else {
+    q.amax_src = x_amax;
+  }
+  NVFP4MOE_TRY(launch_quant(q, s));
+  NVFP4MOE_TRY(mark(2));
+
+  // 4. gate_up grouped GEMM + SwiGLU epilogue (h in BF16, amax of h)
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.q_a = xq;
+  g.sf_a = xsf;
+  g.s_dec_a = xsd;
+  g.s_dec_a_rows = 1;
+  g.q_w = w_gate_up->q;
+  g.sf_w = w_gate_up->sf;
+  g.s_dec_w = w_gate_up->s_dec;
+  g.offsets = offsets;
+  g.padded_offsets = padded;
+  g.E = E;
+  g.rows_cap = cap;
+  g.N = 2 * I;
+  g.K = H;
+  g.epilogue = kEpiSwiGLU;
+  g.out_bf16 = hb;
+  g.out_padded = 1;
+  g.amax_h = tok ? h_amax_rows : h_amax_tensor;
+  g.amax_h_rows = tok ? 1 : 0;
+  g.err = err;
+  NVFP4MOE_TRY(launch_grouped_gemm(g, s));
+  NVFP4MOE_TRY(mark(3));
+
+  // 5. requantize h with the amax the epilogue reduced (amax reuse)
+  QuantParams rq;
+  rq.x = hb;
+  rq.tasks = T * k;
+  rq.K = I;
+  rq.mode = kQuantRequant;
+  rq.amax_src = tok ? h_amax_rows : h_amax_tensor;
+  rq.amax_rows = tok ? 1 : 0;
+  rq.q = hq;
+  rq.sf = hsf;
+  rq.sf_mma = 1;
+  rq.s_dec = hsd;
+  rq.s_dec_rows = 1;
+  rq.rows_cap = cap;
+  rq.offsets = offsets;
+  rq.padded_offsets = padded;
+  rq.E = E;
+  NVFP4MOE_TRY(launch_quant(rq, s));
+  NVFP4MOE_TRY(mark(4));
+
+  // 6. down grouped GEMM -> D (BF16, compact sorted rows)
+  GemmArgs dn;
+  std::memset(&dn, 0, sizeof(dn));
+  dn.q_a = hq;
+  dn.sf_a = hsf;
+  dn.s_dec_a = hsd;
+  dn.s_dec_a_rows = 1;
+  dn.q_w = w_down->q;
+  dn.sf_w = w_down->sf;
+  dn.s_dec_w = w_down->s_dec;
+  dn.offsets = offsets;
+  dn.padded_offsets = padded;
+  dn.E = E;
+  dn.rows_cap = cap;
+  dn.N = H;
+  dn.K = I;
+  dn.epilogue = kEpiStore;
+  dn.out_bf16 = d;
+  dn.out_padded = 0;
+  dn.err = err;
+  NVFP4MOE_TRY(launch_grouped_gemm(dn, s));
+  NVFP4MOE_TRY(mark(5));
+
+  // 7. weighted combine in slot order
+  NVFP4MOE_TRY(launch_combine(d, inv_perm, topk_w, T, k, H, y, s));
+  NVFP4MOE_TRY(mark(6));
+  return NVFP4MOE_OK;
+}
+
+int moe_expert_layer(const void *x, const int32_t *topk_idx, const float *topk_w,
+                     const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down, int64_t T,
+                     int64_t H, int64_t I, int E, int k, void *y, uint32_t flags, void *workspace,
+                     size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  return expert_layer_impl(x, topk_idx, topk_w, w_gate_up, w_down, T, H, I, E, k, y, flags, workspace,
+                           workspace_bytes, stream, nullptr);
+}
+
+int moe_expert_layer_profiled(const void *x, const int32_t *topk_idx, const float *topk_w,
+                              const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down,
+                              int64_t T, int64_t H, int64_t I, int E, int k, void *y, uint32_t flags,
+                              void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream,
+                              void *const *stage_events) {
+  return expert_layer_impl(x, topk_idx, topk_w, w_gate_up, w_down, T, H, I, E, k, y, flags, workspace,
+                           workspace_bytes, stream, stage_events);
+}
+
+int nvfp4moe_encode_e2m1(const float *y, int64_t n, uint8_t *codes, nvfp4moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (y == nullptr || codes == nullptr))) return NVFP4MOE_ERR_INVALID_ARG;
+  return cuda_rc(launch_encode_e2m1(y, n, codes, st(stream)));
+}
+
+int nvfp4moe_encode_ue4m3(const float *v, int64_t n, uint8_t *codes, nvfp4moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (v == nullptr || codes == nullptr))) return NVFP4MOE_ERR_INVALID_ARG;
+  return cuda_rc(launch_encode_ue4m3(v, n, codes, st(stream)));
+}
+
+}  // extern "C"

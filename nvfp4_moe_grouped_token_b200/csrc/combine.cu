@@ -1,0 +1,69 @@
+// Unpermute + top-k weighted combine: y[t] = BF16( sum_j w[t][j] * D[inv_perm[t][j]] ).
+//
+// The sum runs in FP32 in slot order j = 0..k-1 for every token, independent
+// of how the tokens were batched or grouped -- the fixed reduction order the
+// pages' strict-alignment mode needs (news.hamidun.com, "diagnostics,
+// alignment and fast kernels": order of computation is part of the policy).
+//
+// One warp per token; each lane owns 8 consecutive BF16 columns per step
+// (128-bit loads and stores), so a warp moves 512 contiguous bytes per row.
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4moe {
+
+namespace {
+
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    k_combine(const uint4 *__restrict__ d, const int32_t *__restrict__ inv_perm,
+              const float *__restrict__ w, int64_t T, int k, int64_t H, int64_t rows_cap,
+              uint4 *__restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int64_t hv = H >> 3;                 // uint4 per row
+  int32_t my_row = 0;
+  float my_w = 0.0f;
+  if (lane < k) {
+    my_row = __ldg(inv_perm + t * k + lane);
+    my_w = __ldg(w + t * k + lane);
+  }
+  for (int64_t c = lane; c < hv; c += 32) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+      const float wj = __shfl_sync(0xffffffffu, my_w, j);
+      if (row < 0 || row >= rows_cap) continue;   // an invalid routing entry adds nothing
+      const uint4 v = __ldg(d + row * hv + c);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fmaf_rn(wj, bf16_lo(u[i]), acc[2 * i]);
+        acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(u[i]), acc[2 * i + 1]);
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    y[t * hv + c] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const void *d, const int32_t *inv_perm, const float *w, int64_t T, int k,
+                           int64_t H, void *y, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t blocks = (T + kCombineWarps - 1) / kCombineWarps;
+  k_combine<<<(unsigned)blocks, kCombineWarps * 32, 0, s>>>(
+      static_cast<const uint4 *>(d), inv_perm, w, T, k, H, T * k, static_cast<uint4 *>(y));
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

@@ -1,0 +1,105 @@
+// Internal launch interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4moe {
+
+// Where the rows a quantize launch reads come from and where they go.
+enum QuantMode : int {
+  kQuantPlain = 0,     // row i -> row i (nvfp4_quantize)
+  kQuantScatter = 1,   // token t -> its k rows in the padded grouped layout
+  kQuantRequant = 2,   // padded row p of h -> row p (valid rows only)
+  kQuantWeights = 3,   // expert e row n -> expert e row interleave(n)
+};
+
+struct QuantParams {
+  const void *x = nullptr;          // BF16 source
+  int64_t tasks = 0;                // rows (plain), tokens (scatter), T*k (requant), E*N (weights)
+  int64_t K = 0;                    // elements per row
+  int mode = kQuantPlain;
+  // amax: amax_src is the per-tensor value (index 0), per-row values, or per
+  // expert values (weights); amax_rows == 1 means per row.
+  const float *amax_src = nullptr;
+  int amax_rows = 0;
+  int compute_row_amax = 0;         // per-row amax computed here (no amax_src)
+  float *amax_out = nullptr;        // per-row amax written here (per-row modes)
+  // outputs
+  uint8_t *q = nullptr;
+  uint8_t *sf = nullptr;
+  int sf_mma = 0;
+  float *s_dec = nullptr;           // per tensor [1], per row, or per expert
+  int s_dec_rows = 0;               // 1: one S_dec per destination row
+  int64_t rows_cap = 0;             // destination rows allocated (bounds check)
+  // grouped layout (scatter / requant)
+  const int32_t *topk_idx = nullptr;
+  const int32_t *inv_perm = nullptr;    // given positions (standalone scatter)
+  const int32_t *offsets = nullptr;
+  const int32_t *padded_offsets = nullptr;
+  int k = 1;
+  int E = 1;
+  // fused ranks (layer path): positions from per-block bases + local ranks
+  const int32_t *local_rank = nullptr;
+  const int32_t *block_base = nullptr;
+  int32_t *perm_out = nullptr;
+  int32_t *inv_perm_out = nullptr;
+  float *zero_rows = nullptr;       // per-row buffer zeroed at each destination
+  // weights
+  int64_t N = 0;
+  int gate_up = 0;
+  int *err = nullptr;
+};
+
+constexpr int kRankTokens = 128;    // tokens per routing block
+
+cudaError_t launch_amax(const void *x, int64_t seg_len, int64_t nseg, float *out, cudaStream_t s);
+cudaError_t launch_quant(const QuantParams &p, cudaStream_t s);
+cudaError_t launch_encode_e2m1(const float *y, int64_t n, uint8_t *codes, cudaStream_t s);
+cudaError_t launch_encode_ue4m3(const float *v, int64_t n, uint8_t *codes, cudaStream_t s);
+
+struct PermuteParams {
+  const int32_t *topk_idx;
+  int64_t T;
+  int k;
+  int E;
+  int32_t *block_counts;   // [nblk][E]
+  int32_t *local_rank;     // [T*k]
+  int32_t *offsets;        // [E+1]
+  int32_t *padded_offsets; // [E+1]
+  int32_t *perm;           // [T*k] (rank kernel)
+  int32_t *inv_perm;       // [T*k] (rank kernel)
+  int *err;
+};
+int64_t permute_blocks(int64_t T);
+cudaError_t launch_route_count(const PermuteParams &p, cudaStream_t s);
+cudaError_t launch_route_scan(const PermuteParams &p, cudaStream_t s);
+cudaError_t launch_route_rank(const PermuteParams &p, cudaStream_t s);
+
+enum GemmEpilogue : int { kEpiStore = 0, kEpiSwiGLU = 1 };
+
+struct GemmArgs {
+  const uint8_t *q_a, *sf_a;
+  const float *s_dec_a;
+  int s_dec_a_rows;
+  const uint8_t *q_w, *sf_w;
+  const float *s_dec_w;
+  const int32_t *offsets, *padded_offsets;
+  int E;
+  int64_t rows_cap, N, K;
+  int epilogue;
+  void *out_bf16;
+  float *out_f32;
+  int out_padded;
+  float *amax_h;      // SwiGLU: amax of h (per row [rows_cap] or [1])
+  int amax_h_rows;
+  int *err;
+};
+cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
+
+cudaError_t launch_combine(const void *d, const int32_t *inv_perm, const float *w, int64_t T, int k,
+                           int64_t H, void *y, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace nvfp4moe

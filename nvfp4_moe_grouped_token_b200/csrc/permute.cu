@@ -1,0 +1,178 @@
+// Token-to-expert permutation with device-side group offsets.
+//
+// The contiguous per-expert layout and device-side metadata of the token-wise
+// path (www.aib.vote "miniTE report, NVFP4 RL stability", paragraph 4).  Rows
+// are ordered by (expert, token, slot): a stable order that needs no sort and
+// no atomics whose order could vary from run to run.
+//
+//   count  one block per 128 tokens.  Each warp marks, per expert, which of
+//          its 32 tokens chose that expert (a 32-bit mask built with atomicOr,
+//          whose result does not depend on the order of the ORs).  A token's
+//          rank inside its block is the popcount of the masks of the earlier
+//          warps plus that of its own warp below its lane.  Writes the
+//          per-block count of every expert and each (token, slot)'s local rank.
+//   scan   one block: exclusive prefix over blocks per expert (in place), the
+//          expert totals, and their prefix sums -> offsets / padded_offsets.
+//   rank   perm / inv_perm from offsets + block base + local rank (the fused
+//          layer path does this inside the quantize-scatter kernel instead).
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4moe {
+
+namespace {
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kRankTokens) k_route_count(const PermuteParams p) {
+  extern __shared__ uint32_t smem_u[];
+  const int E = p.E, k = p.k;
+  uint32_t *masks = smem_u;                                   // [4][E]
+  int32_t *wpre = reinterpret_cast<int32_t *>(smem_u + 4 * E);  // [4][E]
+  for (int i = threadIdx.x; i < 4 * E; i += blockDim.x) masks[i] = 0;
+  __syncthreads();
+  const int64_t t = (int64_t)blockIdx.x * kRankTokens + threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool live = t < p.T;
+  if (live) {
+    const int32_t *row = p.topk_idx + t * k;
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(row + j);
+      if (e < 0 || e >= E) {
+        set_device_error(p.err, kDevBadExpert, e);
+        continue;
+      }
+      bool dup = false;
+      for (int jj = 0; jj < j; ++jj) dup |= (__ldg(row + jj) == e);
+      if (dup) {
+        set_device_error(p.err, kDevDupExpert, e);
+        continue;
+      }
+      atomicOr(&masks[warp * E + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kRankTokens / 32; ++w) {
+      wpre[w * E + e] = run;
+      run += __popc(masks[w * E + e]);
+    }
+    p.block_counts[(int64_t)blockIdx.x * E + e] = run;
+  }
+  __syncthreads();
+  if (live) {
+    const int32_t *row = p.topk_idx + t * k;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(row + j);
+      int32_t r = -1;
+      if (e >= 0 && e < E) {
+        bool dup = false;
+        for (int jj = 0; jj < j; ++jj) dup |= (__ldg(row + jj) == e);
+        if (!dup) r = wpre[warp * E + e] + __popc(masks[warp * E + e] & below);
+      }
+      p.local_rank[t * k + j] = r;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams p, int64_t nblk) {
+  __shared__ int32_t partial[kScanThreads];
+  __shared__ int32_t scan_a[kScanThreads];
+  __shared__ int32_t scan_b[kScanThreads];
+  const int E = p.E;
+  const int S = kScanThreads / E;          // segments per expert (E <= 1024)
+  const int tid = threadIdx.x;
+  const int e = tid % E, s = tid / E;
+  const int64_t seg = (nblk + S - 1) / S;
+  const int64_t b0 = (int64_t)s * seg;
+  const int64_t b1 = b0 + seg < nblk ? b0 + seg : nblk;
+  int32_t sum = 0;
+  if (s < S) {
+    for (int64_t b = b0; b < b1; ++b) sum += p.block_counts[b * E + e];
+    partial[s * E + e] = sum;
+  }
+  __syncthreads();
+  int32_t total = 0;
+  if (s < S) {
+    int32_t base = 0;
+    for (int ss = 0; ss < S; ++ss) {
+      const int32_t v = partial[ss * E + e];
+      if (ss < s) base += v;
+      total += v;
+    }
+    for (int64_t b = b0; b < b1; ++b) {
+      const int32_t c = p.block_counts[b * E + e];
+      p.block_counts[b * E + e] = base;
+      base += c;
+    }
+  }
+  // inclusive scans of totals and padded totals over experts
+  int32_t v = (tid < E && s == 0) ? total : 0;
+  int32_t vp = (tid < E && s == 0) ? ((total + 127) / 128) * 128 : 0;
+  scan_a[tid] = v;
+  scan_b[tid] = vp;
+  __syncthreads();
+  for (int o = 1; o < kScanThreads; o <<= 1) {
+    const int32_t a = tid >= o ? scan_a[tid - o] : 0;
+    const int32_t b = tid >= o ? scan_b[tid - o] : 0;
+    __syncthreads();
+    scan_a[tid] += a;
+    scan_b[tid] += b;
+    __syncthreads();
+  }
+  if (tid < E) {
+    p.offsets[tid + 1] = scan_a[tid];
+    p.padded_offsets[tid + 1] = scan_b[tid];
+  }
+  if (tid == 0) {
+    p.offsets[0] = 0;
+    p.padded_offsets[0] = 0;
+  }
+}
+
+__global__ void k_route_rank(const PermuteParams p) {
+  const int64_t n = p.T * p.k;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = __ldg(p.topk_idx + i);
+    const int32_t lr = __ldg(p.local_rank + i);
+    if (e < 0 || e >= p.E || lr < 0) continue;
+    const int64_t t = i / p.k;
+    const int64_t r = (int64_t)__ldg(p.offsets + e) +
+                      __ldg(p.block_counts + (t / kRankTokens) * p.E + e) + lr;
+    if (r < 0 || r >= n) continue;
+    p.perm[r] = (int32_t)i;
+    p.inv_perm[i] = (int32_t)r;
+  }
+}
+
+}  // namespace
+
+int64_t permute_blocks(int64_t T) { return (T + kRankTokens - 1) / kRankTokens; }
+
+cudaError_t launch_route_count(const PermuteParams &p, cudaStream_t s) {
+  const int64_t nblk = permute_blocks(p.T);
+  if (nblk == 0) return cudaSuccess;
+  const size_t smem = (size_t)8 * p.E * sizeof(uint32_t);
+  k_route_count<<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_scan(const PermuteParams &p, cudaStream_t s) {
+  k_route_scan<<<1, kScanThreads, 0, s>>>(p, permute_blocks(p.T));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_rank(const PermuteParams &p, cudaStream_t s) {
+  const int64_t n = p.T * p.k;
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  k_route_rank<<<(unsigned)blocks, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

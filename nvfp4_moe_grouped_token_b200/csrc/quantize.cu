@@ -1,0 +1,299 @@
+// NVFP4 quantizer kernels: amax reduction and the row quantizer.
+//
+// The token-wise NVFP4 path (www.aib.vote "miniTE report, NVFP4 RL
+// stability", paragraph 4): every token row is quantized once -- its amax
+// computed once and reused for all of its copies -- and written straight into
+// the contiguous per-expert layout the grouped GEMM reads.
+//
+// One warp owns one row.  Lane l handles the 16-element blocks l, l+32, ...;
+// a block is 32 contiguous bytes of BF16, so a warp reads 1 KB per step with
+// 128-bit coalesced loads, and writes 256 contiguous bytes of codes.  The
+// per-row amax is a warp shuffle reduction; rows of up to 4096 elements stay
+// in registers between the amax pass and the encode pass.
+//
+// Arithmetic per block (one binary32 operation each, round to nearest even):
+//   bamax = max|x|, t = (bamax / 6) * S_enc, sf = UE4M3(t),
+//   r = S_enc / sf, code_i = E2M1(x_i * r); a block with sf == 0 is all +0.
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4moe {
+
+namespace {
+
+constexpr int kQuantWarps = 8;     // rows per 256-thread block
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float abs_max8(uint4 v) {
+  float m = 0.0f;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, fabsf(bf16_lo(w[i])));
+    m = fmaxf(m, fabsf(bf16_hi(w[i])));
+  }
+  return m;
+}
+
+// amax of `nseg` segments of seg_len BF16 each; out[seg] must be 0 beforehand
+// (max of non-negative floats = max of their bit patterns as unsigned).
+__global__ void k_amax(const uint4 *__restrict__ x, int64_t seg_vec, float *__restrict__ out) {
+  const int64_t seg = blockIdx.y;
+  const uint4 *base = x + seg * seg_vec;
+  float m = 0.0f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < seg_vec;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    m = fmaxf(m, abs_max8(__ldg(base + i)));
+  }
+  m = warp_max(m);
+  __shared__ float red[32];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) red[w] = m;
+  __syncthreads();
+  if (w == 0) {
+    m = l < (int)(blockDim.x >> 5) ? red[l] : 0.0f;
+    m = warp_max(m);
+    if (l == 0 && m > 0.0f) atomicMax(reinterpret_cast<unsigned int *>(out + seg), __float_as_uint(m));
+  }
+}
+
+template <int NB>  // 16-element blocks per lane held in registers; 0 = re-read
+__global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t task = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (task >= p.tasks) return;
+  const int64_t K = p.K;
+  const int64_t nblk = K >> 4;
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(p.x);
+
+  // ---- source row, destination row(s), amax source --------------------
+  int64_t src_row = task;
+  int64_t my_dest = -1;          // lane j < ndest holds destination j
+  int ndest = 1;
+  int64_t amax_index = 0;
+  int64_t expert = 0;
+  if (p.mode == kQuantPlain) {
+    my_dest = task;
+    amax_index = p.amax_rows ? task : 0;
+  } else if (p.mode == kQuantScatter) {
+    ndest = p.k;
+    amax_index = p.amax_rows ? task : 0;
+    if (lane < p.k) {
+      const int64_t slot = task * p.k + lane;
+      const int e = __ldg(p.topk_idx + slot);
+      if (p.local_rank != nullptr) p.inv_perm_out[slot] = -1;   // overwritten below when valid
+      if (e >= 0 && e < p.E) {
+        int64_t r;
+        if (p.local_rank != nullptr) {
+          const int64_t blk = task / kRankTokens;
+          const int32_t lr = __ldg(p.local_rank + slot);
+          r = (int64_t)__ldg(p.offsets + e) + __ldg(p.block_base + blk * p.E + e) + lr;
+          if (lr < 0 || r < 0 || r >= p.tasks * p.k) r = -1;
+          if (r >= 0) {
+            p.perm_out[r] = (int32_t)slot;
+            p.inv_perm_out[slot] = (int32_t)r;
+          }
+        } else {
+          r = __ldg(p.inv_perm + slot);
+        }
+        const int64_t pr = r < 0 ? -1 : r - __ldg(p.offsets + e) + __ldg(p.padded_offsets + e);
+        if (pr >= 0 && pr < p.rows_cap) my_dest = pr;
+      }
+    }
+  } else if (p.mode == kQuantRequant) {
+    const int32_t *off = p.offsets;
+    if (task >= (int64_t)__ldg(off + p.E)) return;
+    int lo = 0, hi = p.E;                      // off[lo] <= task < off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((int64_t)__ldg(off + mid) <= task) lo = mid; else hi = mid;
+    }
+    const int64_t pr = task - __ldg(off + lo) + __ldg(p.padded_offsets + lo);
+    if (pr >= p.rows_cap) return;
+    src_row = pr;
+    my_dest = pr;
+    amax_index = p.amax_rows ? pr : 0;
+  } else {  // kQuantWeights
+    expert = task / p.N;
+    const int64_t n = task - expert * p.N;
+    int64_t nd = n;
+    if (p.gate_up) {
+      const int64_t half = p.N >> 1;
+      const int64_t j = n < half ? n : n - half;
+      nd = (j >> 7) * 256 + (n < half ? 0 : 128) + (j & 127);
+    }
+    my_dest = expert * p.N + nd;
+    amax_index = expert;
+  }
+  const uint4 *src = reinterpret_cast<const uint4 *>(xb + src_row * K);
+
+  // ---- amax ------------------------------------------------------------
+  uint4 cache[NB > 0 ? NB : 1][2];
+  float amax;
+  if (p.compute_row_amax) {
+    float m = 0.0f;
+    if constexpr (NB > 0) {
+#pragma unroll
+      for (int c = 0; c < NB; ++c) {
+        const int64_t b = (int64_t)c * 32 + lane;
+        cache[c][0] = make_uint4(0, 0, 0, 0);
+        cache[c][1] = cache[c][0];
+        if (b < nblk) {
+          cache[c][0] = __ldg(src + b * 2);
+          cache[c][1] = __ldg(src + b * 2 + 1);
+          m = fmaxf(m, fmaxf(abs_max8(cache[c][0]), abs_max8(cache[c][1])));
+        }
+      }
+    } else {
+      for (int64_t b = lane; b < nblk; b += 32) {
+        m = fmaxf(m, fmaxf(abs_max8(__ldg(src + b * 2)), abs_max8(__ldg(src + b * 2 + 1))));
+      }
+    }
+    amax = warp_max(m);
+    if (p.amax_out != nullptr && lane == 0) p.amax_out[task] = amax;
+  } else {
+    amax = __ldg(p.amax_src + amax_index);
+  }
+  float s_enc, s_dec;
+  global_scales(amax, s_enc, s_dec);
+
+  // ---- per-destination bookkeeping --------------------------------------
+  if (lane < ndest && my_dest >= 0) {
+    if (p.s_dec_rows) p.s_dec[my_dest] = s_dec;
+    if (p.zero_rows != nullptr) p.zero_rows[my_dest] = 0.0f;
+  }
+  if (!p.s_dec_rows && lane == 0) {
+    if (p.mode == kQuantPlain && task == 0) p.s_dec[0] = s_dec;
+    if (p.mode == kQuantWeights && (task - expert * p.N) == 0) p.s_dec[expert] = s_dec;
+  }
+
+  // ---- encode ------------------------------------------------------------
+  auto encode_chunk = [&](int64_t c, uint4 v0, uint4 v1) {
+    const int64_t b = c * 32 + lane;
+    const bool valid = b < nblk;
+    const float bamax = fmaxf(abs_max8(v0), abs_max8(v1));
+    const float t = __fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc);
+    const uint32_t sfc = cvt_ue4m3(t);
+    uint2 codes = make_uint2(0, 0);
+    if (sfc != 0) {
+      const float r = __fdiv_rn(s_enc, ue4m3_value(sfc));
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        y[2 * i] = __fmul_rn(bf16_lo(w[i]), r);
+        y[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), r);
+      }
+      codes.x = cvt_e2m1x8(y);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        y[2 * i] = __fmul_rn(bf16_lo(w[4 + i]), r);
+        y[2 * i + 1] = __fmul_rn(bf16_hi(w[4 + i]), r);
+      }
+      codes.y = cvt_e2m1x8(y);
+    }
+    // gather the four scales of blocks 4i..4i+3 into lane 4i
+    const int base = lane & ~3;
+    const uint32_t s0 = __shfl_sync(0xffffffffu, sfc, base);
+    const uint32_t s1 = __shfl_sync(0xffffffffu, sfc, base + 1);
+    const uint32_t s2 = __shfl_sync(0xffffffffu, sfc, base + 2);
+    const uint32_t s3 = __shfl_sync(0xffffffffu, sfc, base + 3);
+    const uint32_t sfw = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    for (int d = 0; d < ndest; ++d) {
+      const int64_t row = __shfl_sync(0xffffffffu, my_dest, d);
+      if (row < 0 || !valid) continue;
+      *reinterpret_cast<uint2 *>(p.q + row * (K >> 1) + b * 8) = codes;
+      if ((lane & 3) == 0) {
+        const int64_t off = p.sf_mma ? sf_mma_offset(row, b, K) : row * nblk + b;
+        *reinterpret_cast<uint32_t *>(p.sf + off) = sfw;
+      }
+    }
+  };
+
+  const int64_t nchunks = (nblk + 31) >> 5;
+  if constexpr (NB > 0) {
+#pragma unroll
+    for (int c = 0; c < NB; ++c)
+      if (c < nchunks) encode_chunk(c, cache[c][0], cache[c][1]);
+  } else {
+    for (int64_t c = 0; c < nchunks; ++c) {
+      const int64_t b = c * 32 + lane;
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+      if (b < nblk) {
+        v0 = __ldg(src + b * 2);
+        v1 = __ldg(src + b * 2 + 1);
+      }
+      encode_chunk(c, v0, v1);
+    }
+  }
+}
+
+template <int NB>
+cudaError_t launch_quant_nb(const QuantParams &p, cudaStream_t s) {
+  const int64_t blocks = (p.tasks + kQuantWarps - 1) / kQuantWarps;
+  k_quant<NB><<<(unsigned)blocks, kQuantWarps * 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+__global__ void k_encode_e2m1(const float *__restrict__ y, int64_t n, uint8_t *__restrict__ codes) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float v[8] = {y[i], 0, 0, 0, 0, 0, 0, 0};
+    codes[i] = (uint8_t)(cvt_e2m1x8(v) & 0xFu);
+  }
+}
+
+__global__ void k_encode_ue4m3(const float *__restrict__ v, int64_t n, uint8_t *__restrict__ codes) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    codes[i] = (uint8_t)cvt_ue4m3(v[i]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_amax(const void *x, int64_t seg_len, int64_t nseg, float *out, cudaStream_t s) {
+  if (seg_len <= 0 || nseg <= 0) return cudaSuccess;
+  const int64_t seg_vec = seg_len / 8;
+  int64_t per_seg = (seg_vec + 255) / 256;
+  const int64_t target = (int64_t)num_sms() * 4;
+  int64_t bx = per_seg < target / nseg + 1 ? per_seg : target / nseg + 1;
+  if (bx < 1) bx = 1;
+  dim3 grid((unsigned)bx, (unsigned)nseg);
+  k_amax<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(x), seg_vec, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
+  if (p.tasks <= 0) return cudaSuccess;
+  const int64_t nb = (p.K + 511) / 512;   // 16-element blocks per lane
+  if (!p.compute_row_amax) return launch_quant_nb<0>(p, s);
+  if (nb <= 1) return launch_quant_nb<1>(p, s);
+  if (nb <= 2) return launch_quant_nb<2>(p, s);
+  if (nb <= 4) return launch_quant_nb<4>(p, s);
+  if (nb <= 8) return launch_quant_nb<8>(p, s);
+  return launch_quant_nb<0>(p, s);
+}
+
+cudaError_t launch_encode_e2m1(const float *y, int64_t n, uint8_t *codes, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 65535) blocks = 65535;
+  k_encode_e2m1<<<(unsigned)blocks, 256, 0, s>>>(y, n, codes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_ue4m3(const float *v, int64_t n, uint8_t *codes, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 65535) blocks = 65535;
+  k_encode_ue4m3<<<(unsigned)blocks, 256, 0, s>>>(v, n, codes);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

@@ -1,0 +1,186 @@
+"""The whole W4A4 MoE expert layer on the GPU, checked stage by stage
+(teacher-forced: each stage is recomputed by the oracle from the GPU's own
+previous-stage output), plus the strict-mode batch-invariance check."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe, nvfp4
+from nvfp4_moe_grouped_token_b200 import ops, workloads
+
+from _parity import (check_bf16, check_weights_exact, dequant_weights, gemm_bound, sf_rowmajor,
+                     swiglu_bound)
+
+pytestmark = pytest.mark.gpu
+
+
+class Layer:
+    def __init__(self, cfg, flags):
+        self.cfg = cfg
+        self.flags = flags
+        self.per_token = bool(flags & (ops.SCALE_PER_TOKEN | ops.STRICT))
+        self.inp = workloads.layer_inputs(cfg)
+        self.wgu = ops.nvfp4_prepare_weights(self.inp["w_gate_up"].cuda(), gate_up=True)
+        self.wdn = ops.nvfp4_prepare_weights(self.inp["w_down"].cuda(), gate_up=False)
+        T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+        self.ws = torch.zeros(ops.moe_expert_layer_workspace_size(T, H, I, E, k, flags),
+                              dtype=torch.uint8, device="cuda")
+        self.y = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+        self.x = self.inp["x"].cuda()
+        self.idx = self.inp["topk_idx"].cuda()
+        self.w = self.inp["topk_w"].cuda()
+
+    def run(self):
+        ops.moe_expert_layer(self.x, self.idx, self.w, self.wgu, self.wdn, self.y, self.ws, self.flags)
+        assert ops.device_status(self.ws) == 0
+        c = self.cfg
+        self.v = ops.layer_views(self.ws, c.T, c.H, c.I, c.E, c.k, self.flags)
+
+    def check(self, sample_tokens=None, check_weights=True):
+        c = self.cfg
+        T, H, I, E, k = c.T, c.H, c.I, c.E, c.k
+        v = self.v
+        x = self.inp["x"].float().numpy()
+        idx = self.inp["topk_idx"].numpy()
+        if check_weights:
+            check_weights_exact(self.wgu, self.inp["w_gate_up"], True, experts=range(min(E, 3)))
+            check_weights_exact(self.wdn, self.inp["w_down"], False, experts=range(min(E, 3)))
+        # 1-2. permutation (exact, all rows)
+        info = moe.permutation(idx, E)
+        for key in ("offsets", "padded_offsets", "perm"):
+            assert np.array_equal(v[key].cpu().numpy(), info[key]), key
+        assert np.array_equal(v["inv_perm"].cpu().numpy(), info["inv_perm"])
+        prow = moe.padded_rows(info)
+        tok = info["perm"] // k
+        e_of = moe.expert_of_rows(info["offsets"])
+        # rows under test
+        if sample_tokens is None:
+            rows = np.arange(T * k)
+            toks = np.arange(T)
+        else:
+            toks = np.asarray(sample_tokens)
+            rows = np.sort(info["inv_perm"][toks].reshape(-1))
+        pr = prow[rows]
+        cap = v["rows_cap"]
+        # 3. x quantized once per token, scattered (exact)
+        qx = nvfp4.quantize(x, self.per_token)
+        xq = v["x_q"].cpu().numpy()
+        xsf = sf_rowmajor(v["x_sf"], cap, H)
+        assert np.array_equal(xq[pr], qx["q"][tok[rows]])
+        assert np.array_equal(xsf[pr], qx["sf"][tok[rows]])
+        sd_want = qx["s_dec"][tok[rows]] if self.per_token else np.full(len(rows), qx["s_dec"][0])
+        assert np.array_equal(v["x_sdec"].cpu().numpy()[pr], sd_want)
+        # 4. gate_up + SwiGLU -> h (tolerance, teacher-forced from the exact codes)
+        xh = nvfp4.dequantize(qx["q"], qx["sf"], qx["s_dec"])
+        a = xh[tok[rows]]
+        g = np.empty((len(rows), 2 * I))
+        gs = np.empty_like(g)
+        d_exact = np.empty((len(rows), H))
+        d_abs = np.empty_like(d_exact)
+        h_gpu_all = v["h"].float().cpu().numpy()
+        h_gpu = h_gpu_all[pr]
+        for e in np.unique(e_of[rows]):
+            m = e_of[rows] == e
+            we = dequant_weights(self.wgu, int(e), gate_up=True)
+            g[m] = a[m] @ we.T
+            gs[m] = np.abs(a[m]) @ np.abs(we).T
+        h_exact = moe.swiglu(g, I)
+        tg, tu = gemm_bound(gs[:, :I]), gemm_bound(gs[:, I:])
+        check_bf16(h_gpu, h_exact, swiglu_bound(g[:, :I], g[:, I:], tg, tu), "h")
+        # 5. requant of the GPU's h, amax reused from the epilogue (exact)
+        if self.per_token:
+            qh = nvfp4.quantize(h_gpu, True)
+        else:
+            valid_h = h_gpu_all[prow]                     # every routed row
+            amax = np.abs(valid_h).max()
+            qh = nvfp4.quantize(h_gpu, False, amax_in=np.array([amax], np.float32))
+        hq = v["h_q"].cpu().numpy()
+        hsf = sf_rowmajor(v["h_sf"], cap, I)
+        assert np.array_equal(hq[pr], qh["q"])
+        assert np.array_equal(hsf[pr], qh["sf"])
+        hsd = v["h_sdec"].cpu().numpy()[pr]
+        assert np.array_equal(hsd, qh["s_dec"] if self.per_token else np.full(len(rows), qh["s_dec"][0]))
+        # 6. down GEMM from the GPU's h codes -> D (tolerance)
+        hh = nvfp4.dequantize(qh["q"], qh["sf"], qh["s_dec"])
+        for e in np.unique(e_of[rows]):
+            m = e_of[rows] == e
+            we = dequant_weights(self.wdn, int(e), gate_up=False)
+            d_exact[m] = hh[m] @ we.T
+            d_abs[m] = np.abs(hh[m]) @ np.abs(we).T
+        d_gpu = v["d"].float().cpu().numpy()[rows]
+        check_bf16(d_gpu, d_exact, gemm_bound(d_abs), "D")
+        # 7. combine from the GPU's D (fp32 sum of k terms vs fp64: one BF16 ulp)
+        d_all = v["d"].float().cpu().numpy()
+        inv = info["inv_perm"][toks]
+        wts = self.inp["topk_w"].numpy()[toks].astype(np.float64)
+        y_exact = np.zeros((len(toks), H))
+        for j in range(k):
+            y_exact += wts[:, j:j + 1] * d_all[inv[:, j]]
+        y_gpu = self.y.float().cpu().numpy()[toks]
+        bound = 1e-6 * (np.abs(wts)[:, :, None] * np.abs(d_all[inv])).sum(axis=1) + 1e-30
+        check_bf16(y_gpu, y_exact, bound, "y")
+
+
+SMALL = workloads.LayerConfig("small", T=300, H=256, I=256, E=8, k=2, seed=21)
+
+
+@pytest.mark.parametrize("flags", [0, ops.SCALE_PER_TOKEN, ops.STRICT])
+def test_small_layer_all_rows(flags):
+    L = Layer(SMALL, flags)
+    L.run()
+    L.check()
+
+
+def test_small_layer_end_to_end_against_full_oracle():
+    L = Layer(SMALL, ops.STRICT)
+    L.run()
+    x = L.inp["x"].float().numpy()
+    wgu = moe.QuantWeights(L.inp["w_gate_up"].float().numpy())
+    wdn = moe.QuantWeights(L.inp["w_down"].float().numpy())
+    ref = moe.expert_layer(x, L.inp["topk_idx"].numpy(), L.inp["topk_w"].numpy(), wgu, wdn, per_token=True)
+    y = L.y.float().cpu().numpy()
+    rel = np.linalg.norm(y - ref["y"]) / np.linalg.norm(ref["y"])
+    # not teacher-forced: requant code flips near rounding boundaries are expected
+    print(f"end-to-end relative L2 difference vs oracle: {rel:.3g}")
+    assert rel < 2e-2
+
+
+def test_moe30b_layer_sampled():
+    cfg = workloads.CONFIGS["moe30b"]
+    L = Layer(cfg, 0)
+    L.run()
+    L.check(sample_tokens=np.arange(0, cfg.T, 509), check_weights=False)
+
+
+def test_dense4b_layer_sampled():
+    cfg = workloads.CONFIGS["dense4b"]
+    L = Layer(cfg, ops.SCALE_PER_TOKEN)
+    L.run()
+    L.check(sample_tokens=np.arange(0, cfg.T, 1021), check_weights=False)
+
+
+def test_strict_batch_invariance():
+    """Each token's BF16 output is bitwise identical whether the 4096 tokens
+    run as one batch, as batches of 1, 7 and 64, or in a shuffled order."""
+    cfg = workloads.CONFIGS["strict"]
+    L = Layer(cfg, ops.STRICT)
+    L.run()
+    full = L.y.clone()
+    T = cfg.T
+
+    def run_subset(tok_idx):
+        n = len(tok_idx)
+        y = torch.empty(n, cfg.H, dtype=torch.bfloat16, device="cuda")
+        ops.moe_expert_layer(L.x[tok_idx], L.idx[tok_idx], L.w[tok_idx], L.wgu, L.wdn, y, L.ws, ops.STRICT)
+        return y
+
+    for bs in (1, 7, 64):
+        out = torch.empty_like(full)
+        for s in range(0, T, bs):
+            sl = torch.arange(s, min(s + bs, T), device="cuda")
+            out[sl] = run_subset(sl)
+        assert torch.equal(out.view(torch.int16), full.view(torch.int16)), f"batch size {bs}"
+    order = torch.randperm(T, generator=torch.Generator().manual_seed(5)).cuda()
+    shuffled = run_subset(order)
+    assert torch.equal(shuffled.view(torch.int16), full[order].view(torch.int16)), "shuffled order"
+    assert ops.device_status(L.ws) == 0
