@@ -135,6 +135,28 @@ def stage_bytes(cfg, counts_pad_rows: int) -> dict:
     }
 
 
+# ------------------------------------------------------- multi-rank ----
+
+def rank_config(cfg, rank: int, world: int):
+    """Data-parallel replicas: every rank runs the same layer shape on its own
+    tokens (seed shifted by rank), with a full copy of the weights."""
+    return cfg if world == 1 else workloads.scaled(cfg, seed=cfg.seed + 1000 * rank)
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's time (the job's time) via all_reduce(MAX)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
 # --------------------------------------------------------------- ours ----
 
 def run_ours(args, rank, world, local_rank):
@@ -142,9 +164,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = workloads.CONFIGS[args.config]
-    if world > 1:
-        cfg = workloads.scaled(cfg, seed=cfg.seed + 1000 * rank)   # each rank its own tokens
+    cfg = rank_config(workloads.CONFIGS[args.config], rank, world)
     flags = 0 if args.per_tensor else ops.SCALE_PER_TOKEN
     inp = workloads.layer_inputs(cfg)
     x = inp["x"].to(dev)
@@ -195,11 +215,7 @@ def run_ours(args, rank, world, local_rank):
     step_ms = [evs[i][0].elapsed_time(evs[i][nstage]) for i in range(args.steps)]
     stage_ms = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                 for j, name in enumerate(ops.STAGES)}
-    ms = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(total_ms / args.steps, world, dev)
 
     # ---- end to end through the public API with host buffers ----------------
     xh = inp["x"].pin_memory()
@@ -225,11 +241,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
 
     fl = layer_flops(cfg)
     pk = peaks()
@@ -240,7 +252,7 @@ def run_ours(args, rank, world, local_rank):
     sb = stage_bytes(cfg, 0)
     result = {
         "metric": METRIC,
-        "value": world * cfg.T / (ms * 1e-3),
+        "value": job_throughput(cfg.T, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -271,7 +283,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": gu_tflops / fp4_peak_sustained,
                      "peak_note": f"{pk['source']} sustained bf16 x {FP4_PER_BF16:g} (nominal FP4:BF16 ratio)",
                      "traffic": traffic},
-        "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(cfg.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4,
                 "d2h_bytes_per_step": yh.numel() * 2},
         "gpu_launches": args.steps * (7 + (1 if args.per_tensor else 0)),

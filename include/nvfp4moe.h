@@ -262,6 +262,32 @@ int nvfp4moe_encode_e2m1(const float *y, int64_t n, uint8_t *codes,
 int nvfp4moe_encode_ue4m3(const float *v, int64_t n, uint8_t *codes,
                           nvfp4moe_stream_t stream);
 
+/* Tensor-core throughput probe: `grid` CTAs (one per SM when grid equals the
+ * SM count) each issue `iters` K-steps of 4 block-scaled FP4 MMAs
+ * (tcgen05.mma kind::mxf4nvf4, M = 128, N = n in {128, 256}, K = 64) on
+ * operands resident in shared memory, each K-step preceded by sf_a_copies
+ * (0..4) and sf_b_copies (0..8) 512-byte scale-factor copies into TMEM, as
+ * the grouped GEMM issues them.  Reads no global memory; cycles[grid]
+ * (device, int64) receives each CTA's elapsed SM cycles.  The FLOP count is
+ * grid * iters * 4 * 2*128*n*64.  mode: 0 = a K-step's copies then its
+ * MMAs; 1 = each K-block's copies right before its MMA; 2 = the copies of
+ * the next K-step (into a second TMEM buffer) before the current MMAs;
+ * 3 = copies only; 4 = mode 0 with 4 + 8 copies issued from precomputed
+ * descriptors; 5 = those copies only; 6 = four 2 KB 128x128b copies only;
+ * 7 = four 1 KB 64x128b.warpx2 copies only; 8 = four warps write 48 scale
+ * columns per K-step with tcgen05.st, no MMAs; 9 = mode 8 alongside the
+ * MMAs of mode 0 without copies; 10 / 11 = modes 8 / 9 with the 48 words
+ * per lane first read from the 6 KB of scale atoms in shared memory; 12 = the
+ * MMAs of mode 0 while another warp fills 54 KB of shared memory per K-step
+ * with bulk copies from global memory.  workspace: 16 bytes (error word),
+ * 256 + 55296 bytes for mode 12 (the bulk copies' source). */
+int nvfp4moe_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies,
+                       int mode, int grid, long long *cycles, void *workspace,
+                       nvfp4moe_stream_t stream);
+
+/* Number of SMs of the current device (the persistent grids' size). */
+int nvfp4moe_num_sms(void);
+
 #ifdef __cplusplus
 }
 #endif

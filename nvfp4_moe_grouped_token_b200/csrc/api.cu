@@ -283,7 +283,8 @@ int nvfp4_grouped_gemm(const uint8_t *q_a, const uint8_t *sf_a, const float *s_d
                        int64_t N, int64_t K, void *out_bf16, float *out_f32, uint32_t flags,
                        void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream) {
   if (E < 1 || rows_cap < 0 || N <= 0 || K <= 0) return NVFP4MOE_ERR_INVALID_ARG;
-  if (K % 256 != 0 || N % 256 != 0 || rows_cap % 128 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (K % 256 != 0 || N % 256 != 0 || rows_cap % 128 != 0 || E > 1024)
+    return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
   if (q_a == nullptr || sf_a == nullptr || s_dec_a == nullptr || q_w == nullptr || sf_w == nullptr ||
       s_dec_w == nullptr || offsets == nullptr || padded_offsets == nullptr ||
       (out_bf16 == nullptr && out_f32 == nullptr))
@@ -562,6 +563,20 @@ int moe_expert_layer_profiled(const void *x, const int32_t *topk_idx, const floa
   return expert_layer_impl(x, topk_idx, topk_w, w_gate_up, w_down, T, H, I, E, k, y, flags, workspace,
                            workspace_bytes, stream, stage_events);
 }
+
+int nvfp4moe_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies, int mode, int grid,
+                       long long *cycles, void *workspace, nvfp4moe_stream_t stream) {
+  if (iters < 1 || (n != 128 && n != 256) || sf_a_copies < 0 || sf_a_copies > 4 || sf_b_copies < 0 ||
+      sf_b_copies > 8 || mode < 0 || mode > 12 || grid < 1 || cycles == nullptr || workspace == nullptr)
+    return NVFP4MOE_ERR_INVALID_ARG;
+  cudaStream_t s = st(stream);
+  NVFP4MOE_TRY(cudaMemsetAsync(workspace, 0, 16, s));
+  return cuda_rc(launch_mma_probe(iters, n, sf_a_copies, sf_b_copies, mode, cycles,
+                                  static_cast<int *>(workspace),
+                                  static_cast<const uint8_t *>(workspace) + 256, grid, s));
+}
+
+int nvfp4moe_num_sms(void) { return num_sms(); }
 
 int nvfp4moe_encode_e2m1(const float *y, int64_t n, uint8_t *codes, nvfp4moe_stream_t stream) {
   if (n < 0 || (n > 0 && (y == nullptr || codes == nullptr))) return NVFP4MOE_ERR_INVALID_ARG;

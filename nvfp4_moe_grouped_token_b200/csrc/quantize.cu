@@ -8,8 +8,8 @@
 // One warp owns one row.  Lane l handles the 16-element blocks l, l+32, ...;
 // a block is 32 contiguous bytes of BF16, so a warp reads 1 KB per step with
 // 128-bit coalesced loads, and writes 256 contiguous bytes of codes.  The
-// per-row amax is a warp shuffle reduction; rows of up to 4096 elements stay
-// in registers between the amax pass and the encode pass.
+// per-row amax is a warp shuffle reduction; rows of up to 4096 elements are
+// loaded into registers up front, before the amax is known.
 //
 // Arithmetic per block (one binary32 operation each, round to nearest even):
 //   bamax = max|x|, t = (bamax / 6) * S_enc, sf = UE4M3(t),
@@ -132,23 +132,26 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   }
   const uint4 *src = reinterpret_cast<const uint4 *>(xb + src_row * K);
 
-  // ---- amax ------------------------------------------------------------
+  // ---- load the row (registers when it fits), then its amax -------------
   uint4 cache[NB > 0 ? NB : 1][2];
+  if constexpr (NB > 0) {
+#pragma unroll
+    for (int c = 0; c < NB; ++c) {
+      const int64_t b = (int64_t)c * 32 + lane;
+      cache[c][0] = make_uint4(0, 0, 0, 0);
+      cache[c][1] = cache[c][0];
+      if (b < nblk) {
+        cache[c][0] = __ldg(src + b * 2);
+        cache[c][1] = __ldg(src + b * 2 + 1);
+      }
+    }
+  }
   float amax;
   if (p.compute_row_amax) {
     float m = 0.0f;
     if constexpr (NB > 0) {
 #pragma unroll
-      for (int c = 0; c < NB; ++c) {
-        const int64_t b = (int64_t)c * 32 + lane;
-        cache[c][0] = make_uint4(0, 0, 0, 0);
-        cache[c][1] = cache[c][0];
-        if (b < nblk) {
-          cache[c][0] = __ldg(src + b * 2);
-          cache[c][1] = __ldg(src + b * 2 + 1);
-          m = fmaxf(m, fmaxf(abs_max8(cache[c][0]), abs_max8(cache[c][1])));
-        }
-      }
+      for (int c = 0; c < NB; ++c) m = fmaxf(m, fmaxf(abs_max8(cache[c][0]), abs_max8(cache[c][1])));
     } else {
       for (int64_t b = lane; b < nblk; b += 32) {
         m = fmaxf(m, fmaxf(abs_max8(__ldg(src + b * 2)), abs_max8(__ldg(src + b * 2 + 1))));
@@ -233,6 +236,101 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   }
 }
 
+// Requantization of h, one thread per 16-element block (the row's amax is
+// known: the GEMM epilogue reduced it).  A CTA takes `rpb` consecutive
+// routed rows; the per-row facts (padded row, S_enc, S_dec) are resolved
+// once per row into shared memory, then every thread encodes one block:
+// 32 bytes read, 8 bytes of codes and one scale written.  No lane idles on a
+// ragged row (K = 768 has 48 blocks, 1.5 warps).
+__global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, int rpb) {
+  extern __shared__ int32_t sm[];
+  const int E = p.E;
+  int32_t *s_off = sm;                       // [E+1]
+  int32_t *s_pad = sm + (E + 1);             // [E+1]
+  int64_t *s_row = reinterpret_cast<int64_t *>(sm + 2 * (E + 1));   // [rpb], 8-byte aligned
+  float *s_enc_r = reinterpret_cast<float *>(s_row + rpb);                         // [rpb]
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+    s_off[i] = __ldg(p.offsets + i);
+    s_pad[i] = __ldg(p.padded_offsets + i);
+  }
+  __syncthreads();
+  const int64_t K = p.K;
+  const int nblk = (int)(K >> 4);
+  const int64_t R = s_off[E];
+  const int64_t r0 = (int64_t)blockIdx.x * rpb;
+  if (threadIdx.x < rpb) {
+    const int64_t r = r0 + threadIdx.x;
+    int64_t pr = -1;
+    float se = 1.0f;
+    if (r < R) {
+      int lo = 0, hi = E;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)s_off[mid] <= r) lo = mid; else hi = mid;
+      }
+      pr = r - s_off[lo] + s_pad[lo];
+      if (pr >= p.rows_cap) pr = -1;
+      if (pr >= 0) {
+        float sd;
+        global_scales(__ldg(p.amax_src + (p.amax_rows ? pr : 0)), se, sd);
+        p.s_dec[pr] = sd;
+      }
+    }
+    s_row[threadIdx.x] = pr;
+    s_enc_r[threadIdx.x] = se;
+  }
+  __syncthreads();
+  const int rl = threadIdx.x / nblk;
+  const int b = threadIdx.x - rl * nblk;
+  const int64_t pr = rl < rpb ? s_row[rl] : -1;
+  const bool valid = pr >= 0;
+  uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+  if (valid) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + pr * K) + b * 2;
+    v0 = __ldg(src);
+    v1 = __ldg(src + 1);
+  }
+  const float s_enc = valid ? s_enc_r[rl] : 1.0f;
+  // block amax on packed BF16 pairs (exact: a max of BF16 values)
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i])));
+  const float bamax = fmaxf(__low2float(m2), __high2float(m2));
+  const float t = __fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc);
+  const uint32_t sfc = valid ? cvt_ue4m3(t) : 0u;
+  uint2 codes = make_uint2(0, 0);
+  if (sfc != 0) {
+    const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      y[2 * i] = __fmul_rn(bf16_lo(w[i]), rr);
+      y[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), rr);
+    }
+    codes.x = cvt_e2m1x8(y);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      y[2 * i] = __fmul_rn(bf16_lo(w[4 + i]), rr);
+      y[2 * i + 1] = __fmul_rn(bf16_hi(w[4 + i]), rr);
+    }
+    codes.y = cvt_e2m1x8(y);
+  }
+  // four consecutive blocks of one row sit in lanes 4i..4i+3 (rows start at
+  // multiples of nblk, a multiple of 4)
+  const int lane = threadIdx.x & 31;
+  const int base = lane & ~3;
+  const uint32_t s0 = __shfl_sync(0xffffffffu, sfc, base);
+  const uint32_t s1 = __shfl_sync(0xffffffffu, sfc, base + 1);
+  const uint32_t s2 = __shfl_sync(0xffffffffu, sfc, base + 2);
+  const uint32_t s3 = __shfl_sync(0xffffffffu, sfc, base + 3);
+  if (valid) {
+    *reinterpret_cast<uint2 *>(p.q + pr * (K >> 1) + (int64_t)b * 8) = codes;
+    if ((lane & 3) == 0)
+      *reinterpret_cast<uint32_t *>(p.sf + sf_mma_offset(pr, b, K)) = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
 template <int NB>
 cudaError_t launch_quant_nb(const QuantParams &p, cudaStream_t s) {
   const int64_t blocks = (p.tasks + kQuantWarps - 1) / kQuantWarps;
@@ -271,8 +369,16 @@ cudaError_t launch_amax(const void *x, int64_t seg_len, int64_t nseg, float *out
 
 cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
   if (p.tasks <= 0) return cudaSuccess;
+  if (p.mode == kQuantRequant && !p.compute_row_amax && p.K / 16 <= 256 && p.sf_mma) {
+    const int nblk = (int)(p.K / 16);
+    const int rpb = 256 / nblk;                       // rows per CTA
+    const int threads = ((rpb * nblk + 31) / 32) * 32;
+    const size_t smem = (size_t)8 * (p.E + 2) + (size_t)12 * rpb + 16;
+    const int64_t blocks = (p.tasks + rpb - 1) / rpb;
+    k_requant_blocks<<<(unsigned)blocks, threads, smem, s>>>(p, rpb);
+    return cudaGetLastError();
+  }
   const int64_t nb = (p.K + 511) / 512;   // 16-element blocks per lane
-  if (!p.compute_row_amax) return launch_quant_nb<0>(p, s);
   if (nb <= 1) return launch_quant_nb<1>(p, s);
   if (nb <= 2) return launch_quant_nb<2>(p, s);
   if (nb <= 4) return launch_quant_nb<4>(p, s);

@@ -61,6 +61,8 @@ _SIGS = {
                                          _vp, _u32, _vp, _sz, _vp, ctypes.POINTER(_vp)]),
     "nvfp4moe_encode_e2m1": (_i32, [_vp, _i64, _vp, _vp]),
     "nvfp4moe_encode_ue4m3": (_i32, [_vp, _i64, _vp, _vp]),
+    "nvfp4moe_mma_probe": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "nvfp4moe_num_sms": (_i32, []),
 }
 
 _LIB = None
@@ -268,6 +270,30 @@ def nvfp4moe_encode_e2m1(y: torch.Tensor, codes: torch.Tensor, stream=None):
 def nvfp4moe_encode_ue4m3(v: torch.Tensor, codes: torch.Tensor, stream=None):
     _dev(v, codes)
     _check(lib().nvfp4moe_encode_ue4m3(_p(v), v.numel(), _p(codes), _stream(stream)), "encode_ue4m3")
+
+
+def mma_probe(iters: int, n: int = 256, sf_a_copies: int = 4, sf_b_copies: int = 8, mode: int = 0,
+              grid: int = 0, stream=None) -> dict:
+    """nvfp4moe_mma_probe: dense block-scaled FP4 MMA throughput on this GPU.
+    Returns TFLOP/s (from CUDA events) and FLOP per SM per cycle."""
+    grid = grid or lib().nvfp4moe_num_sms()
+    cyc = torch.zeros(grid, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(256 + 55296, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream() if stream is None else stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    _check(lib().nvfp4moe_mma_probe(iters, n, sf_a_copies, sf_b_copies, mode, grid, _p(cyc), _p(ws),
+                                    _stream(stream)), "nvfp4moe_mma_probe")
+    e1.record(s)
+    torch.cuda.synchronize()
+    if device_status(ws) != OK:
+        raise NVFP4Error("mma probe wait timed out")
+    flop = grid * iters * 4 * 2.0 * 128 * n * 64
+    ms = e0.elapsed_time(e1)
+    c = cyc.float().mean().item()
+    return {"tflops": flop / (ms * 1e-3) / 1e12, "flop_per_sm_cycle": flop / grid / c, "ms": ms,
+            "cycles_mean": c, "grid": grid, "n": n, "sf_a_copies": sf_a_copies, "sf_b_copies": sf_b_copies,
+            "mode": mode}
 
 
 # ------------------------------------------------------------------ helpers --
