@@ -129,6 +129,23 @@ int moe_permute(const int32_t *topk_idx, int64_t T, int k, int E,
                 int32_t *inv_perm, void *workspace, size_t workspace_bytes,
                 nvfp4moe_stream_t stream);
 
+/* moe_permute for callers that cannot provide any scratch memory -- code
+ * inside a host framework whose memory planner owns all device memory and
+ * allows no allocation after start-up, or code running where cudaMalloc is
+ * not allowed.  The pages have no counterpart of this entry point.
+ * Same arguments and outputs as moe_permute, without the workspace: the
+ * scratch is a static device array of the library (about 1 MB per GPU that
+ * loads it, held until the process exits).  Limits: T*k <= 131072 and
+ * ceil(T/128)*E <= 131072 (NVFP4MOE_ERR_WORKSPACE beyond them).  It allocates
+ * nothing; its first call on a device looks up the array's address (make that
+ * call before any stream capture).  Calls that overlap on the GPU race on the
+ * shared array.  Bad or duplicate expert ids are skipped as in moe_permute
+ * but not reported (there is no workspace error word to read). */
+int moe_permute_noalloc(const int32_t *topk_idx, int64_t T, int k, int E,
+                        int32_t *offsets, int32_t *padded_offsets,
+                        int32_t *perm, int32_t *inv_perm,
+                        nvfp4moe_stream_t stream);
+
 /* Quantize each token of x [T][K] once and write its codes, scales and
  * decode scale to all k of its rows in the padded grouped layout (the fused
  * quantize + permute of the token-wise path: amax computed once, reused for

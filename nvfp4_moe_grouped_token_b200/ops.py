@@ -45,6 +45,7 @@ _SIGS = {
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _u32, _vp]),
     "moe_permute_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_quantize_permute": (_i32, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _i64, _u32, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64,
@@ -142,6 +143,14 @@ def moe_permute(topk_idx, E, offsets, padded_offsets, perm, inv_perm, workspace,
     _check(lib().moe_permute(_p(topk_idx), T, k, E, _p(offsets), _p(padded_offsets), _p(perm),
                              _p(inv_perm), _p(workspace), workspace.numel() * workspace.element_size(),
                              _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(topk_idx, E, offsets, padded_offsets, perm, inv_perm, stream=None):
+    """moe_permute with the library's static scratch: no workspace argument."""
+    _dev(topk_idx, offsets, padded_offsets, perm, inv_perm)
+    T, k = topk_idx.shape
+    _check(lib().moe_permute_noalloc(_p(topk_idx), T, k, E, _p(offsets), _p(padded_offsets), _p(perm),
+                                     _p(inv_perm), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_quantize_permute(x, topk_idx, inv_perm, offsets, padded_offsets, E, q_rows, sf_rows,
