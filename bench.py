@@ -293,14 +293,24 @@ def run_ours(args, rank, world, local_rank):
 
 
 def load_traffic(kernel_key: str):
-    """DRAM bytes per launch from the committed ncu summary, if present and current."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    """DRAM bytes per launch of a GEMM launch from profiles/traffic.txt (one ncu
+    capture), or None when the kernel source changed since that capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "nvfp4_moe_grouped_token_b200", "csrc", "gemm.cu")
+    if not os.path.exists(path) or not os.path.exists(src):
         return None
+    vals = {}
     with open(path) as f:
-        d = json.load(f)
-    v = d.get(kernel_key)
-    return None if v is None else v.get("dram_bytes_per_launch")
+        for line in f:
+            parts = line.split()
+            if len(parts) == 2 and not line.startswith("#"):
+                vals[parts[0]] = parts[1]
+    with open(src, "rb") as f:
+        if hashlib.sha1(f.read()).hexdigest() != vals.get("gemm_sha1"):
+            return None
+    v = vals.get(kernel_key)
+    return None if v is None else int(v)
 
 
 # ------------------------------------------------------- oracle (CPU) ----
