@@ -29,15 +29,13 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// max |x| of 8 BF16 values on packed pairs (exact: a max of BF16 values)
 __device__ __forceinline__ float abs_max8(uint4 v) {
-  float m = 0.0f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  __nv_bfloat162 m = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = fmaxf(m, fabsf(bf16_lo(w[i])));
-    m = fmaxf(m, fabsf(bf16_hi(w[i])));
-  }
-  return m;
+  for (int i = 1; i < 4; ++i) m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i])));
+  return fmaxf(__low2float(m), __high2float(m));
 }
 
 // amax of `nseg` segments of seg_len BF16 each; out[seg] must be 0 beforehand
@@ -71,13 +69,46 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   const int64_t nblk = K >> 4;
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(p.x);
 
-  // ---- source row, destination row(s), amax source --------------------
+  // ---- source row ----------------------------------------------------------
   int64_t src_row = task;
   int64_t my_dest = -1;          // lane j < ndest holds destination j
   int ndest = 1;
   int64_t amax_index = 0;
   int64_t expert = 0;
-  if (p.mode == kQuantPlain) {
+  if (p.mode == kQuantRequant) {
+    const int32_t *off = p.offsets;
+    if (task >= (int64_t)__ldg(off + p.E)) return;
+    int lo = 0, hi = p.E;                      // off[lo] <= task < off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((int64_t)__ldg(off + mid) <= task) lo = mid; else hi = mid;
+    }
+    const int64_t pr = task - __ldg(off + lo) + __ldg(p.padded_offsets + lo);
+    if (pr >= p.rows_cap) return;
+    src_row = pr;
+    my_dest = pr;
+    amax_index = p.amax_rows ? pr : 0;
+  }
+  const uint4 *src = reinterpret_cast<const uint4 *>(xb + src_row * K);
+
+  // ---- load the row (registers when it fits) before anything that waits ---
+  uint4 cache[NB > 0 ? NB : 1][2];
+  if constexpr (NB > 0) {
+#pragma unroll
+    for (int c = 0; c < NB; ++c) {
+      const int64_t b = (int64_t)c * 32 + lane;
+      cache[c][0] = make_uint4(0, 0, 0, 0);
+      cache[c][1] = cache[c][0];
+      if (b < nblk) {
+        cache[c][0] = __ldg(src + b * 2);
+        cache[c][1] = __ldg(src + b * 2 + 1);
+      }
+    }
+  }
+
+  // ---- destination row(s), amax source ----------------------------------
+  if (p.mode == kQuantRequant) {
+  } else if (p.mode == kQuantPlain) {
     my_dest = task;
     amax_index = p.amax_rows ? task : 0;
   } else if (p.mode == kQuantScatter) {
@@ -105,19 +136,6 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
         if (pr >= 0 && pr < p.rows_cap) my_dest = pr;
       }
     }
-  } else if (p.mode == kQuantRequant) {
-    const int32_t *off = p.offsets;
-    if (task >= (int64_t)__ldg(off + p.E)) return;
-    int lo = 0, hi = p.E;                      // off[lo] <= task < off[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if ((int64_t)__ldg(off + mid) <= task) lo = mid; else hi = mid;
-    }
-    const int64_t pr = task - __ldg(off + lo) + __ldg(p.padded_offsets + lo);
-    if (pr >= p.rows_cap) return;
-    src_row = pr;
-    my_dest = pr;
-    amax_index = p.amax_rows ? pr : 0;
   } else {  // kQuantWeights
     expert = task / p.N;
     const int64_t n = task - expert * p.N;
@@ -130,22 +148,8 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
     my_dest = expert * p.N + nd;
     amax_index = expert;
   }
-  const uint4 *src = reinterpret_cast<const uint4 *>(xb + src_row * K);
 
-  // ---- load the row (registers when it fits), then its amax -------------
-  uint4 cache[NB > 0 ? NB : 1][2];
-  if constexpr (NB > 0) {
-#pragma unroll
-    for (int c = 0; c < NB; ++c) {
-      const int64_t b = (int64_t)c * 32 + lane;
-      cache[c][0] = make_uint4(0, 0, 0, 0);
-      cache[c][1] = cache[c][0];
-      if (b < nblk) {
-        cache[c][0] = __ldg(src + b * 2);
-        cache[c][1] = __ldg(src + b * 2 + 1);
-      }
-    }
-  }
+  // ---- amax ---------------------------------------------------------------
   float amax;
   if (p.compute_row_amax) {
     float m = 0.0f;
@@ -236,66 +240,41 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   }
 }
 
-// Requantization of h, one thread per 16-element block (the row's amax is
-// known: the GEMM epilogue reduced it).  A CTA takes `rpb` consecutive
-// routed rows; the per-row facts (padded row, S_enc, S_dec) are resolved
-// once per row into shared memory, then every thread encodes one block:
-// 32 bytes read, 8 bytes of codes and one scale written.  No lane idles on a
-// ragged row (K = 768 has 48 blocks, 1.5 warps).
-__global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, int rpb) {
-  extern __shared__ int32_t sm[];
-  const int E = p.E;
-  int32_t *s_off = sm;                       // [E+1]
-  int32_t *s_pad = sm + (E + 1);             // [E+1]
-  int64_t *s_row = reinterpret_cast<int64_t *>(sm + 2 * (E + 1));   // [rpb], 8-byte aligned
-  float *s_enc_r = reinterpret_cast<float *>(s_row + rpb);                         // [rpb]
-  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
-    s_off[i] = __ldg(p.offsets + i);
-    s_pad[i] = __ldg(p.padded_offsets + i);
-  }
-  __syncthreads();
+// Requantization of h, one thread per 16-element block of a routed row (the
+// row's amax is known: the GEMM epilogue reduced it).  Thread i takes routed
+// row r = i / nblk, block i % nblk; it finds the row's padded position from
+// the L1-resident group offsets (no CTA-wide setup, no barrier) and loads its
+// 32 bytes of h and the row's amax.  No lane idles on a ragged row (K = 768
+// is 48 blocks, 1.5 warps).
+__global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, uint32_t nblk, uint32_t total) {
+  // 32-bit index math: a 64-bit division is a long software sequence
+  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
   const int64_t K = p.K;
-  const int nblk = (int)(K >> 4);
-  const int64_t R = s_off[E];
-  const int64_t r0 = (int64_t)blockIdx.x * rpb;
-  if (threadIdx.x < rpb) {
-    const int64_t r = r0 + threadIdx.x;
-    int64_t pr = -1;
-    float se = 1.0f;
-    if (r < R) {
-      int lo = 0, hi = E;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)s_off[mid] <= r) lo = mid; else hi = mid;
-      }
-      pr = r - s_off[lo] + s_pad[lo];
-      if (pr >= p.rows_cap) pr = -1;
-      if (pr >= 0) {
-        float sd;
-        global_scales(__ldg(p.amax_src + (p.amax_rows ? pr : 0)), se, sd);
-        p.s_dec[pr] = sd;
-      }
-    }
-    s_row[threadIdx.x] = pr;
-    s_enc_r[threadIdx.x] = se;
+  const uint32_t r = i / nblk;
+  const int b = (int)(i - r * nblk);
+  const int32_t *off = p.offsets;
+  const int64_t R = __ldg(off + p.E);
+  bool valid = i < total && (int64_t)r < R;
+  int lo = 0, hi = p.E;                              // off[lo] <= r < off[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)__ldg(off + mid) <= (int64_t)r) lo = mid; else hi = mid;
   }
-  __syncthreads();
-  const int rl = threadIdx.x / nblk;
-  const int b = threadIdx.x - rl * nblk;
-  const int64_t pr = rl < rpb ? s_row[rl] : -1;
-  const bool valid = pr >= 0;
-  uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-  if (valid) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + pr * K) + b * 2;
-    v0 = __ldg(src);
-    v1 = __ldg(src + 1);
-  }
-  const float s_enc = valid ? s_enc_r[rl] : 1.0f;
+  int64_t pr = (int64_t)r - __ldg(off + lo) + __ldg(p.padded_offsets + lo);
+  if (pr < 0 || pr >= p.rows_cap) valid = false;
+  if (!valid) pr = 0;
+  const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + pr * K) + b * 2;
+  const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+  const float amax = __ldg(p.amax_src + (p.amax_rows ? pr : 0));
+  float s_enc, s_dec;
+  global_scales(amax, s_enc, s_dec);
+  if (valid && b == 0) p.s_dec[pr] = s_dec;
   // block amax on packed BF16 pairs (exact: a max of BF16 values)
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
   __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
 #pragma unroll
-  for (int i = 1; i < 8; ++i) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i])));
+  for (int j = 1; j < 8; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
   const float bamax = fmaxf(__low2float(m2), __high2float(m2));
   const float t = __fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc);
   const uint32_t sfc = valid ? cvt_ue4m3(t) : 0u;
@@ -304,21 +283,21 @@ __global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, int
     const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
     float y[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      y[2 * i] = __fmul_rn(bf16_lo(w[i]), rr);
-      y[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), rr);
+    for (int j = 0; j < 4; ++j) {
+      y[2 * j] = __fmul_rn(bf16_lo(w[j]), rr);
+      y[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), rr);
     }
     codes.x = cvt_e2m1x8(y);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      y[2 * i] = __fmul_rn(bf16_lo(w[4 + i]), rr);
-      y[2 * i + 1] = __fmul_rn(bf16_hi(w[4 + i]), rr);
+    for (int j = 0; j < 4; ++j) {
+      y[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), rr);
+      y[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), rr);
     }
     codes.y = cvt_e2m1x8(y);
   }
-  // four consecutive blocks of one row sit in lanes 4i..4i+3 (rows start at
-  // multiples of nblk, a multiple of 4)
-  const int lane = threadIdx.x & 31;
+  // four consecutive blocks of one row sit in lanes 4i..4i+3 (a row starts at
+  // a multiple of nblk, itself a multiple of 4, and 256-thread CTAs start at
+  // multiples of 4 too)
   const int base = lane & ~3;
   const uint32_t s0 = __shfl_sync(0xffffffffu, sfc, base);
   const uint32_t s1 = __shfl_sync(0xffffffffu, sfc, base + 1);
@@ -369,13 +348,12 @@ cudaError_t launch_amax(const void *x, int64_t seg_len, int64_t nseg, float *out
 
 cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
   if (p.tasks <= 0) return cudaSuccess;
-  if (p.mode == kQuantRequant && !p.compute_row_amax && p.K / 16 <= 256 && p.sf_mma) {
-    const int nblk = (int)(p.K / 16);
-    const int rpb = 256 / nblk;                       // rows per CTA
-    const int threads = ((rpb * nblk + 31) / 32) * 32;
-    const size_t smem = (size_t)8 * (p.E + 2) + (size_t)12 * rpb + 16;
-    const int64_t blocks = (p.tasks + rpb - 1) / rpb;
-    k_requant_blocks<<<(unsigned)blocks, threads, smem, s>>>(p, rpb);
+  if (p.mode == kQuantRequant && !p.compute_row_amax && p.sf_mma) {
+    const uint32_t nblk = (uint32_t)(p.K / 16);
+    const int64_t total = p.tasks * nblk;             // every routed row (T*k bound), every block
+    if (total >= (int64_t)1 << 31) return cudaErrorInvalidValue;
+    const int64_t blocks = (total + 255) / 256;
+    k_requant_blocks<<<(unsigned)blocks, 256, 0, s>>>(p, nblk, (uint32_t)total);
     return cudaGetLastError();
   }
   const int64_t nb = (p.K + 511) / 512;   // 16-element blocks per lane
