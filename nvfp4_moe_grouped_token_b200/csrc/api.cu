@@ -437,6 +437,9 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   pp.perm = perm;
   pp.inv_perm = inv_perm;
   pp.err = err;
+  // padding rows of h start with amax 0 (the requantizer skips them)
+  pp.zero_pad_rows = tok ? h_amax_rows : nullptr;
+  pp.rows_cap = cap;
   NVFP4MOE_TRY(launch_route_count(pp, s));
   if (!tok) NVFP4MOE_TRY(launch_amax(x, T * H, 1, x_amax, s));
   NVFP4MOE_TRY(launch_route_scan(pp, s));

@@ -70,6 +70,10 @@ struct PermuteParams {
   int32_t *perm;           // [T*k] (rank kernel)
   int32_t *inv_perm;       // [T*k] (rank kernel)
   int *err;
+  // optional: per-row floats zeroed on every padding row [padded start + count,
+  // padded end) of each group below rows_cap (scan kernel)
+  float *zero_pad_rows = nullptr;
+  int64_t rows_cap = 0;
 };
 int64_t permute_blocks(int64_t T);
 cudaError_t launch_route_count(const PermuteParams &p, cudaStream_t s);

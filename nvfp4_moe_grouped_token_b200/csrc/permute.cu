@@ -131,6 +131,12 @@ __global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams
     p.offsets[0] = 0;
     p.padded_offsets[0] = 0;
   }
+  if (p.zero_pad_rows != nullptr && tid < E) {
+    const int64_t end = scan_b[tid];
+    int64_t r = end - vp + v;                // first padding row of the group
+    const int64_t stop = end < p.rows_cap ? end : p.rows_cap;
+    for (; r < stop; ++r) p.zero_pad_rows[r] = 0.0f;
+  }
 }
 
 __global__ void k_route_rank(const PermuteParams p) {

@@ -60,7 +60,10 @@ __global__ void k_amax(const uint4 *__restrict__ x, int64_t seg_vec, float *__re
   }
 }
 
-template <int NB>  // 16-element blocks per lane held in registers; 0 = re-read
+// NB: 16-element blocks per lane held in registers (0 = re-read).
+// KD > 0: at most KD destination rows whose byte offsets fit 32 bits, kept in
+// registers for the whole row; KD == 0: any number, looked up per store.
+template <int NB, int KD>
 __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t task = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
@@ -179,6 +182,21 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
     if (p.mode == kQuantWeights && (task - expert * p.N) == 0) p.s_dec[expert] = s_dec;
   }
 
+  // ---- destination offsets (codes, scale row part) ------------------------
+  uint32_t qoff[KD > 0 ? KD : 1], soff[KD > 0 ? KD : 1];
+  bool dvalid[KD > 0 ? KD : 1];
+  if constexpr (KD > 0) {
+#pragma unroll
+    for (int d = 0; d < KD; ++d) {
+      const int64_t row = __shfl_sync(0xffffffffu, my_dest, d);
+      dvalid[d] = d < ndest && row >= 0;
+      const uint32_t r32 = dvalid[d] ? (uint32_t)row : 0u;
+      qoff[d] = r32 * (uint32_t)(K >> 1);
+      soff[d] = p.sf_mma ? ((r32 >> 7) * (uint32_t)(K >> 6) * 512u + (r32 & 31u) * 16u + ((r32 & 127u) >> 5) * 4u)
+                         : r32 * (uint32_t)nblk;
+    }
+  }
+
   // ---- encode ------------------------------------------------------------
   auto encode_chunk = [&](int64_t c, uint4 v0, uint4 v1) {
     const int64_t b = c * 32 + lane;
@@ -211,13 +229,24 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
     const uint32_t s2 = __shfl_sync(0xffffffffu, sfc, base + 2);
     const uint32_t s3 = __shfl_sync(0xffffffffu, sfc, base + 3);
     const uint32_t sfw = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
-    for (int d = 0; d < ndest; ++d) {
-      const int64_t row = __shfl_sync(0xffffffffu, my_dest, d);
-      if (row < 0 || !valid) continue;
-      *reinterpret_cast<uint2 *>(p.q + row * (K >> 1) + b * 8) = codes;
-      if ((lane & 3) == 0) {
-        const int64_t off = p.sf_mma ? sf_mma_offset(row, b, K) : row * nblk + b;
-        *reinterpret_cast<uint32_t *>(p.sf + off) = sfw;
+    if constexpr (KD > 0) {
+      const uint32_t qb = (uint32_t)b * 8u;
+      const uint32_t sb = p.sf_mma ? ((uint32_t)b >> 2) * 512u : (uint32_t)b;
+#pragma unroll
+      for (int d = 0; d < KD; ++d) {
+        if (!dvalid[d] || !valid) continue;
+        *reinterpret_cast<uint2 *>(p.q + qoff[d] + qb) = codes;
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(p.sf + soff[d] + sb) = sfw;
+      }
+    } else {
+      for (int d = 0; d < ndest; ++d) {
+        const int64_t row = __shfl_sync(0xffffffffu, my_dest, d);
+        if (row < 0 || !valid) continue;
+        *reinterpret_cast<uint2 *>(p.q + row * (K >> 1) + b * 8) = codes;
+        if ((lane & 3) == 0) {
+          const int64_t off = p.sf_mma ? sf_mma_offset(row, b, K) : row * nblk + b;
+          *reinterpret_cast<uint32_t *>(p.sf + off) = sfw;
+        }
       }
     }
   };
@@ -240,80 +269,96 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   }
 }
 
-// Requantization of h, one thread per 16-element block of a routed row (the
-// row's amax is known: the GEMM epilogue reduced it).  Thread i takes routed
-// row r = i / nblk, block i % nblk; it finds the row's padded position from
-// the L1-resident group offsets (no CTA-wide setup, no barrier) and loads its
-// 32 bytes of h and the row's amax.  No lane idles on a ragged row (K = 768
-// is 48 blocks, 1.5 warps).
-__global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, uint32_t nblk, uint32_t total) {
-  // 32-bit index math: a 64-bit division is a long software sequence
-  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+// Requantization of the padded rows of h with the amax the GEMM epilogue
+// reduced (amax reuse): thread per 16-element block, grid-stride over the
+// padded rows [0, padded_offsets[E]) so no lane searches the group offsets.
+// A row whose amax is 0 -- a padding row (the route scan zeroes their amax) or
+// an all-zero row -- gets zero codes, zero scales and S_dec = 1, exactly what
+// quantizing a zero row gives, without reading h.  (r, b) of a lane advance by
+// the fixed stride, so the loop divides once.
+__global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, uint32_t nblk) {
   const int lane = threadIdx.x & 31;
   const int64_t K = p.K;
-  const uint32_t r = i / nblk;
-  const int b = (int)(i - r * nblk);
-  const int32_t *off = p.offsets;
-  const int64_t R = __ldg(off + p.E);
-  bool valid = i < total && (int64_t)r < R;
-  int lo = 0, hi = p.E;                              // off[lo] <= r < off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if ((int64_t)__ldg(off + mid) <= (int64_t)r) lo = mid; else hi = mid;
-  }
-  int64_t pr = (int64_t)r - __ldg(off + lo) + __ldg(p.padded_offsets + lo);
-  if (pr < 0 || pr >= p.rows_cap) valid = false;
-  if (!valid) pr = 0;
-  const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + pr * K) + b * 2;
-  const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-  const float amax = __ldg(p.amax_src + (p.amax_rows ? pr : 0));
-  float s_enc, s_dec;
-  global_scales(amax, s_enc, s_dec);
-  if (valid && b == 0) p.s_dec[pr] = s_dec;
-  // block amax on packed BF16 pairs (exact: a max of BF16 values)
-  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
+  int64_t rows = __ldg(p.padded_offsets + p.E);
+  if (rows > p.rows_cap) rows = p.rows_cap;
+  if (rows < 0) rows = 0;
+  const uint32_t total = (uint32_t)rows * nblk;
+  const uint32_t stride = gridDim.x * blockDim.x;        // a multiple of 32
+  const uint32_t step_r = stride / nblk, step_b = stride - step_r * nblk;
+  uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t r = i / nblk, b = i - r * nblk;
+  // warp-uniform trip count: the shuffles below need every lane
+  for (uint32_t base = i - lane; base < total; base += stride) {
+    const bool valid = i < total;
+    const float amax = valid ? __ldg(p.amax_src + (p.amax_rows ? r : 0)) : 0.0f;
+    float s_enc = 1.0f, s_dec = 1.0f;
+    uint32_t sfc = 0;
+    uint2 codes = make_uint2(0, 0);
+    if (amax > 0.0f) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) +
+                                                         (int64_t)r * K) + b * 2;
+      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      global_scales(amax, s_enc, s_dec);
+      // block amax on packed BF16 pairs (exact: a max of BF16 values)
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
 #pragma unroll
-  for (int j = 1; j < 8; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
-  const float bamax = fmaxf(__low2float(m2), __high2float(m2));
-  const float t = __fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc);
-  const uint32_t sfc = valid ? cvt_ue4m3(t) : 0u;
-  uint2 codes = make_uint2(0, 0);
-  if (sfc != 0) {
-    const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
-    float y[8];
+      for (int j = 1; j < 8; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
+      const float bamax = fmaxf(__low2float(m2), __high2float(m2));
+      sfc = cvt_ue4m3(__fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc));
+      if (sfc != 0) {
+        const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
+        float y[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      y[2 * j] = __fmul_rn(bf16_lo(w[j]), rr);
-      y[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), rr);
+        for (int j = 0; j < 4; ++j) {
+          y[2 * j] = __fmul_rn(bf16_lo(w[j]), rr);
+          y[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), rr);
+        }
+        codes.x = cvt_e2m1x8(y);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          y[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), rr);
+          y[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), rr);
+        }
+        codes.y = cvt_e2m1x8(y);
+      }
     }
-    codes.x = cvt_e2m1x8(y);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      y[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), rr);
-      y[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), rr);
+    // four consecutive blocks of one row sit in lanes 4i..4i+3 (rows start at
+    // multiples of nblk, itself a multiple of 4, and the stride and warp
+    // bases are multiples of 32)
+    const int q4 = lane & ~3;
+    const uint32_t s0 = __shfl_sync(0xffffffffu, sfc, q4);
+    const uint32_t s1 = __shfl_sync(0xffffffffu, sfc, q4 + 1);
+    const uint32_t s2 = __shfl_sync(0xffffffffu, sfc, q4 + 2);
+    const uint32_t s3 = __shfl_sync(0xffffffffu, sfc, q4 + 3);
+    if (valid) {
+      if (b == 0) p.s_dec[r] = s_dec;
+      *reinterpret_cast<uint2 *>(p.q + (int64_t)r * (K >> 1) + (int64_t)b * 8) = codes;
+      if ((lane & 3) == 0)
+        *reinterpret_cast<uint32_t *>(p.sf + sf_mma_offset(r, b, K)) = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
-    codes.y = cvt_e2m1x8(y);
-  }
-  // four consecutive blocks of one row sit in lanes 4i..4i+3 (a row starts at
-  // a multiple of nblk, itself a multiple of 4, and 256-thread CTAs start at
-  // multiples of 4 too)
-  const int base = lane & ~3;
-  const uint32_t s0 = __shfl_sync(0xffffffffu, sfc, base);
-  const uint32_t s1 = __shfl_sync(0xffffffffu, sfc, base + 1);
-  const uint32_t s2 = __shfl_sync(0xffffffffu, sfc, base + 2);
-  const uint32_t s3 = __shfl_sync(0xffffffffu, sfc, base + 3);
-  if (valid) {
-    *reinterpret_cast<uint2 *>(p.q + pr * (K >> 1) + (int64_t)b * 8) = codes;
-    if ((lane & 3) == 0)
-      *reinterpret_cast<uint32_t *>(p.sf + sf_mma_offset(pr, b, K)) = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    i += stride;
+    r += step_r;
+    b += step_b;
+    if (b >= nblk) {
+      b -= nblk;
+      ++r;
+    }
   }
 }
 
 template <int NB>
 cudaError_t launch_quant_nb(const QuantParams &p, cudaStream_t s) {
   const int64_t blocks = (p.tasks + kQuantWarps - 1) / kQuantWarps;
-  k_quant<NB><<<(unsigned)blocks, kQuantWarps * 32, 0, s>>>(p);
+  // every mode writes rows below rows_cap; 32-bit byte offsets when they fit
+  const int ndest = p.mode == kQuantScatter ? p.k : 1;
+  const bool small = p.rows_cap * (p.K >> 1) < ((int64_t)1 << 31);
+  if (small && ndest <= 1)
+    k_quant<NB, 1><<<(unsigned)blocks, kQuantWarps * 32, 0, s>>>(p);
+  else if (small && ndest <= 8)
+    k_quant<NB, 8><<<(unsigned)blocks, kQuantWarps * 32, 0, s>>>(p);
+  else
+    k_quant<NB, 0><<<(unsigned)blocks, kQuantWarps * 32, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -350,10 +395,13 @@ cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
   if (p.tasks <= 0) return cudaSuccess;
   if (p.mode == kQuantRequant && !p.compute_row_amax && p.sf_mma) {
     const uint32_t nblk = (uint32_t)(p.K / 16);
-    const int64_t total = p.tasks * nblk;             // every routed row (T*k bound), every block
-    if (total >= (int64_t)1 << 31) return cudaErrorInvalidValue;
-    const int64_t blocks = (total + 255) / 256;
-    k_requant_blocks<<<(unsigned)blocks, 256, 0, s>>>(p, nblk, (uint32_t)total);
+    // every padded row below rows_cap, every block; 32-bit indices
+    if (p.rows_cap * (int64_t)nblk >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    int64_t blocks = (p.rows_cap * nblk + 255) / 256;
+    const int64_t persistent = (int64_t)num_sms() * 8;  // 8 CTAs of 256 threads per SM
+    if (blocks > persistent) blocks = persistent;
+    if (blocks < 1) blocks = 1;
+    k_requant_blocks<<<(unsigned)blocks, 256, 0, s>>>(p, nblk);
     return cudaGetLastError();
   }
   const int64_t nb = (p.K + 511) / 512;   // 16-element blocks per lane
