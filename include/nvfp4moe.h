@@ -25,6 +25,11 @@
  *                 byte(row, b) = ((row/128)*(K/64) + b/4)*512 + (row%32)*16
  *                                + ((row%128)/32)*4 + b%4
  *                 (rows of a matrix padded to a multiple of 128).
+ *   K-step-major  the activations' layout in the padded grouped layout:
+ *                 byte(row, b) = ((b/16)*rows_cap + row)*16 + b%16, i.e.
+ *                 [K/256][rows_cap][16] -- the 16 scales of a row's 256-element
+ *                 K-step are contiguous, and a 128-row tile's scales for one
+ *                 K-step are 2 KB contiguous (one bulk copy for the GEMM).
  *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless the comment says host.  The caller
@@ -151,7 +156,7 @@ int moe_permute_noalloc(const int32_t *topk_idx, int64_t T, int k, int E,
  * quantize + permute of the token-wise path: amax computed once, reused for
  * every copy).  Uses the inv_perm / offsets / padded_offsets of moe_permute.
  *   q_rows      [rows_cap][K/2] codes at padded row positions (out)
- *   sf_rows     MMA-layout scales over rows_cap rows (out)
+ *   sf_rows     scales in the K-step-major layout (out)
  *   s_dec_rows  [rows_cap] FP32 per-row decode scale (out; per-tensor mode
  *               writes the tensor's S_dec into every row)
  *   amax_in / amax_out as for nvfp4_quantize (per tensor [1], per token [T])
@@ -173,7 +178,7 @@ int moe_quantize_permute(const void *x, int64_t T, int64_t K, int k, int E,
  * with a, w the block-scaled E2M1 values; FP32 accumulation in the tensor
  * cores, one rounding to the output type.
  *   q_a, sf_a, s_dec_a  A in the padded grouped layout (moe_quantize_permute):
- *                       q_a [rows_cap][K/2], sf_a MMA layout, s_dec_a
+ *                       q_a [rows_cap][K/2], sf_a K-step-major, s_dec_a
  *                       [rows_cap] (NVFP4MOE_SCALE_PER_TOKEN) or [1]
  *   q_w, sf_w, s_dec_w  weights: q_w [E][N][K/2], sf_w MMA layout per expert
  *                       ([E][N/128][K/64][512] bytes), s_dec_w [E]

@@ -161,7 +161,7 @@ int nvfp4_quantize(const void *x, int64_t M, int64_t K, const float *amax_in, fl
   p.mode = kQuantPlain;
   p.q = q;
   p.sf = scales;
-  p.sf_mma = (flags & NVFP4MOE_SF_MMA_LAYOUT) ? 1 : 0;
+  p.sf_layout = (flags & NVFP4MOE_SF_MMA_LAYOUT) ? kSfMma : kSfRowMajor;
   p.s_dec = s_dec;
   p.s_dec_rows = tok ? 1 : 0;
   p.rows_cap = M;
@@ -247,7 +247,7 @@ int moe_quantize_permute(const void *x, int64_t T, int64_t K, int k, int E, cons
   p.mode = kQuantScatter;
   p.q = q_rows;
   p.sf = sf_rows;
-  p.sf_mma = 1;
+  p.sf_layout = kSfKStep;
   p.s_dec = s_dec_rows;
   p.s_dec_rows = 1;
   p.rows_cap = rows_cap;
@@ -340,7 +340,7 @@ int nvfp4_prepare_weights(const void *w, int64_t E, int64_t N, int64_t K, uint32
   p.amax_rows = 1;
   p.q = out->q;
   p.sf = out->sf;
-  p.sf_mma = 1;
+  p.sf_layout = kSfMma;
   p.s_dec = out->s_dec;
   p.s_dec_rows = 0;
   p.rows_cap = E * N;
@@ -453,7 +453,7 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   q.mode = kQuantScatter;
   q.q = xq;
   q.sf = xsf;
-  q.sf_mma = 1;
+  q.sf_layout = kSfKStep;
   q.s_dec = xsd;
   q.s_dec_rows = 1;
   q.rows_cap = cap;
@@ -511,7 +511,7 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   rq.amax_rows = tok ? 1 : 0;
   rq.q = hq;
   rq.sf = hsf;
-  rq.sf_mma = 1;
+  rq.sf_layout = kSfKStep;
   rq.s_dec = hsd;
   rq.s_dec_rows = 1;
   rq.rows_cap = cap;

@@ -13,10 +13,12 @@
 //     slower for down: twice the A re-reads).  A rows come
 //     from the padded grouped layout, where every expert's group starts on a
 //     128-row boundary, so a tile never straddles two experts.
-//   * warp 0, one thread: TMA producer.  Per K-step it loads the A tile
-//     (16 KB) and the B tile (32 KB) with 128-byte-swizzled tensor copies and
-//     the scale factors (2 KB + 4 KB, already stored in the MMA atom layout)
-//     with plain bulk copies, into a shared-memory ring.
+//   * warp 4, one thread: TMA producer.  Per K-step it loads the A tile
+//     (16 KB) and the B tile (32 KB) with 128-byte-swizzled tensor copies,
+//     and the scales with plain bulk copies: A's 2 KB (the K-step-major
+//     layout [K/256][rows][16] puts a tile's 128 rows x 16 scales of one
+//     K-step in one contiguous run) and B's 4 KB (prepared in the MMA atom
+//     layout), into a shared-memory ring.
 //   * warp 1, one thread: copies the scale factors into TMEM (tcgen05.cp) and
 //     issues tcgen05.mma kind::mxf4nvf4 with 16-element UE4M3 scale blocks,
 //     FP32 accumulators in TMEM (256 columns), then commits the stage back to
@@ -196,12 +198,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   if (warp < kFeedWarps) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsFeed));
     // --------------------------------------------------------- feeders
-    // For every K-step: wait for the stage's TMA data, read this warp's
-    // lanes' 16-byte records of the 4 SFA and 4*kNAtoms SFB scale atoms from
-    // shared memory and write them into the stage's TMEM scale slot with
-    // tcgen05.st (the MMA reads scales from TMEM).  tcgen05.st runs an order
-    // of magnitude faster than tcgen05.cp for these small atoms and overlaps
-    // the MMAs.
+    // For every K-step: wait for the stage's TMA data, build this lane's
+    // records of the stage's scales and write them into the stage's TMEM
+    // scale slot with tcgen05.st (the MMA reads scales from TMEM).  The slot
+    // holds the MMA atom layout: for K-block group kb (4 scale blocks), lane i
+    // of every 32-lane quarter carries rows i, i+32, i+64, i+96.  A's scales
+    // arrive as 128 rows x 16 bytes, so lane i reads those four 16-byte rows
+    // and the 4x4 word transpose is a register renaming; B's arrive as atoms.  tcgen05.st
+    // runs an order of magnitude faster than tcgen05.cp for these small
+    // copies and overlaps the MMAs.
     const uint32_t tq = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t st = 0, ph = 0;
     for (uint32_t g = 0; g < steps; ++g, st = (st + 1 == STAGES) ? 0 : st + 1, ph ^= (st == 0)) {
@@ -212,9 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       const uint4 *sfb = sfa + C::kSfaBytes / 16;
       uint32_t w[C::kSfSlotCols];
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        const uint4 v = sfa[kb * 32 + lane];
-        w[4 * kb] = v.x; w[4 * kb + 1] = v.y; w[4 * kb + 2] = v.z; w[4 * kb + 3] = v.w;
+      for (int j = 0; j < 4; ++j) {          // row lane + 32 j: 16 scales = word kb for group kb
+        const uint4 v = sfa[j * 32 + lane];
+        w[j] = v.x; w[4 + j] = v.y; w[8 + j] = v.z; w[12 + j] = v.w;
       }
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
@@ -249,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
         const int e = find_group(s_pad, a.E, mt * BM);
         const int32_t arow = (int32_t)(mt * BM);
         const int32_t wrow0 = (int32_t)((int64_t)e * a.N + (int64_t)nt * BN);
-        const uint8_t *sfa_src = a.sf_a + mt * k_atoms * 512;
+        const uint8_t *sfa_src = a.sf_a + mt * BM * 16;   // K-step 0 of the tile's rows
+        const int64_t sfa_step = a.rows_cap * 16;           // one K-step further
         const uint8_t *sfb_src = a.sf_w + ((int64_t)e * (a.N >> 7) + C::kNAtoms * nt) * k_atoms * 512;
         const int64_t sfb_h = k_atoms * 512;
         uint32_t st = p % STAGES, ph = (p / STAGES) & 1u;
@@ -260,11 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
           tma_load_2d(sb, &P.tmap_a, kt * (BK / 2), arow, &full[st]);
           tma_load_2d(sb + C::kABytes, &P.tmap_b, kt * (BK / 2), wrow0, &full[st]);
           bulk_load(sb + C::kABytes + C::kBBytes, sfa_src, C::kSfaBytes, &full[st]);
+          sfa_src += sfa_step;
 #pragma unroll
           for (int h = 0; h < C::kNAtoms; ++h)
             bulk_load(sb + C::kABytes + C::kBBytes + C::kSfaBytes + h * 2048, sfb_src + h * sfb_h, 2048,
                       &full[st]);
-          sfa_src += C::kSfaBytes;
           sfb_src += 2048;
           if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
@@ -500,6 +506,7 @@ cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
   if (!encode_2d(&P.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_w, (uint64_t)(a.K / 2),
                  (uint64_t)(a.E * a.N), BK / 2, C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+
   std::memset(&P.tmap_out, 0, sizeof(P.tmap_out));
   if (a.out_bf16 != nullptr) {
     // D: [rows][N] (compact rows never exceed rows_cap); h: [rows_cap][N/2]

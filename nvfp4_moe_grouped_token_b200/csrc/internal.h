@@ -14,6 +14,14 @@ enum QuantMode : int {
   kQuantWeights = 3,   // expert e row n -> expert e row interleave(n)
 };
 
+// Byte layouts of a scale matrix (one UE4M3 byte per 16 elements along K):
+//   kSfRowMajor  [rows][K/16]
+//   kSfMma       the 128-row x 4-scale atoms the block-scaled MMA reads
+//   kSfKStep     [K/256][rows_cap][16]: the 16 scales of one 256-element
+//                K-step of a row are 16 contiguous bytes, and the scales of
+//                128 consecutive rows for one K-step are 2 KB contiguous
+enum SfLayout : int { kSfRowMajor = 0, kSfMma = 1, kSfKStep = 2 };
+
 struct QuantParams {
   const void *x = nullptr;          // BF16 source
   int64_t tasks = 0;                // rows (plain), tokens (scatter), T*k (requant), E*N (weights)
@@ -28,7 +36,7 @@ struct QuantParams {
   // outputs
   uint8_t *q = nullptr;
   uint8_t *sf = nullptr;
-  int sf_mma = 0;
+  int sf_layout = 0;                // SfLayout
   float *s_dec = nullptr;           // per tensor [1], per row, or per expert
   int s_dec_rows = 0;               // 1: one S_dec per destination row
   int64_t rows_cap = 0;             // destination rows allocated (bounds check)

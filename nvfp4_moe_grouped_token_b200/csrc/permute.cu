@@ -131,11 +131,19 @@ __global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams
     p.offsets[0] = 0;
     p.padded_offsets[0] = 0;
   }
-  if (p.zero_pad_rows != nullptr && tid < E) {
-    const int64_t end = scan_b[tid];
-    int64_t r = end - vp + v;                // first padding row of the group
-    const int64_t stop = end < p.rows_cap ? end : p.rows_cap;
-    for (; r < stop; ++r) p.zero_pad_rows[r] = 0.0f;
+  if (p.zero_pad_rows != nullptr) {
+    // a warp per group: its at most 127 padding rows in four 32-wide steps
+    __syncthreads();
+    if (tid < E) scan_a[tid] = v;            // counts again (the scan is done with scan_a)
+    __syncthreads();
+    const int lane = tid & 31;
+    for (int g = tid >> 5; g < E; g += kScanThreads / 32) {
+      const int64_t end = scan_b[g];
+      const int32_t cnt = scan_a[g];
+      const int64_t start = end - (((int64_t)cnt + 127) / 128) * 128;
+      const int64_t stop = end < p.rows_cap ? end : p.rows_cap;
+      for (int64_t r = start + cnt + lane; r < stop; r += 32) p.zero_pad_rows[r] = 0.0f;
+    }
   }
 }
 

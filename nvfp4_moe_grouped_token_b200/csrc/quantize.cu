@@ -38,6 +38,13 @@ __device__ __forceinline__ float abs_max8(uint4 v) {
   return fmaxf(__low2float(m), __high2float(m));
 }
 
+// Byte offset of scale (row, block b) in the given SfLayout.
+__device__ __forceinline__ int64_t sf_offset(int layout, int64_t row, int64_t b, int64_t K, int64_t rows_cap) {
+  if (layout == kSfMma) return sf_mma_offset(row, b, K);
+  if (layout == kSfKStep) return ((b >> 4) * rows_cap + row) * 16 + (b & 15);
+  return row * (K >> 4) + b;
+}
+
 // amax of `nseg` segments of seg_len BF16 each; out[seg] must be 0 beforehand
 // (max of non-negative floats = max of their bit patterns as unsigned).
 __global__ void k_amax(const uint4 *__restrict__ x, int64_t seg_vec, float *__restrict__ out) {
@@ -192,8 +199,10 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
       dvalid[d] = d < ndest && row >= 0;
       const uint32_t r32 = dvalid[d] ? (uint32_t)row : 0u;
       qoff[d] = r32 * (uint32_t)(K >> 1);
-      soff[d] = p.sf_mma ? ((r32 >> 7) * (uint32_t)(K >> 6) * 512u + (r32 & 31u) * 16u + ((r32 & 127u) >> 5) * 4u)
-                         : r32 * (uint32_t)nblk;
+      soff[d] = p.sf_layout == kSfMma ? ((r32 >> 7) * (uint32_t)(K >> 6) * 512u + (r32 & 31u) * 16u +
+                                         ((r32 & 127u) >> 5) * 4u)
+                : p.sf_layout == kSfKStep ? r32 * 16u
+                                          : r32 * (uint32_t)nblk;
     }
   }
 
@@ -231,7 +240,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
     const uint32_t sfw = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
     if constexpr (KD > 0) {
       const uint32_t qb = (uint32_t)b * 8u;
-      const uint32_t sb = p.sf_mma ? ((uint32_t)b >> 2) * 512u : (uint32_t)b;
+      const uint32_t sb = p.sf_layout == kSfMma ? ((uint32_t)b >> 2) * 512u
+                          : p.sf_layout == kSfKStep ? ((uint32_t)b >> 4) * (uint32_t)p.rows_cap * 16u + ((uint32_t)b & 15u)
+                                                    : (uint32_t)b;
 #pragma unroll
       for (int d = 0; d < KD; ++d) {
         if (!dvalid[d] || !valid) continue;
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
         if (row < 0 || !valid) continue;
         *reinterpret_cast<uint2 *>(p.q + row * (K >> 1) + b * 8) = codes;
         if ((lane & 3) == 0) {
-          const int64_t off = p.sf_mma ? sf_mma_offset(row, b, K) : row * nblk + b;
+          const int64_t off = sf_offset(p.sf_layout, row, b, K, p.rows_cap);
           *reinterpret_cast<uint32_t *>(p.sf + off) = sfw;
         }
       }
@@ -335,7 +346,8 @@ __global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, uin
       if (b == 0) p.s_dec[r] = s_dec;
       *reinterpret_cast<uint2 *>(p.q + (int64_t)r * (K >> 1) + (int64_t)b * 8) = codes;
       if ((lane & 3) == 0)
-        *reinterpret_cast<uint32_t *>(p.sf + sf_mma_offset(r, b, K)) = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        *reinterpret_cast<uint32_t *>(p.sf + sf_offset(p.sf_layout, r, b, K, p.rows_cap)) =
+            s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
     i += stride;
     r += step_r;
@@ -393,7 +405,7 @@ cudaError_t launch_amax(const void *x, int64_t seg_len, int64_t nseg, float *out
 
 cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
   if (p.tasks <= 0) return cudaSuccess;
-  if (p.mode == kQuantRequant && !p.compute_row_amax && p.sf_mma) {
+  if (p.mode == kQuantRequant && !p.compute_row_amax) {
     const uint32_t nblk = (uint32_t)(p.K / 16);
     // every padded row below rows_cap, every block; 32-bit indices
     if (p.rows_cap * (int64_t)nblk >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;

@@ -336,6 +336,13 @@ def layer_views(workspace: torch.Tensor, T, H, I, E, k, flags=0) -> dict:
     }
 
 
+def sf_kstep_to_rowmajor(sf_flat: torch.Tensor, rows_cap: int, K: int) -> torch.Tensor:
+    """Rearrange scales stored in the K-step-major layout of the padded grouped
+    layout ([K/256][rows_cap][16]) into row-major [rows_cap][K/16]."""
+    a = sf_flat[: rows_cap * (K // 16)].view(K // 256, rows_cap, 16)
+    return a.permute(1, 0, 2).reshape(rows_cap, K // 16)
+
+
 def sf_mma_to_rowmajor(sf_flat: torch.Tensor, rows: int, K: int) -> torch.Tensor:
     """Rearrange scales stored in the MMA atom layout into row-major
     [rows][K/16] (an index permutation; used to compare layouts in tests)."""

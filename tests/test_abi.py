@@ -87,6 +87,18 @@ def test_layer_rejects_unsupported_shapes():
     assert lay(P16, P16, P16, ctypes.byref(w), ctypes.byref(wd2), 8, 256, 256, 4, 2, P16, 0, P16, 1 << 30, None) == -3
 
 
+def test_sf_kstep_layout_matches_its_definition():
+    import torch
+    cap, K = 384, 512
+    flat = torch.arange(cap * K // 16, dtype=torch.int64)
+    rm = ops.sf_kstep_to_rowmajor(flat, cap, K)
+    assert rm.shape == (cap, K // 16)
+    assert torch.equal(torch.sort(rm.reshape(-1)).values, flat)
+    # byte(row, b) = ((b/16)*rows_cap + row)*16 + b%16, as the header defines it
+    for row, b in [(0, 0), (5, 3), (200, 17), (383, 31)]:
+        assert int(rm[row, b]) == ((b // 16) * cap + row) * 16 + b % 16
+
+
 def test_sf_layout_permutation_is_a_bijection():
     import torch
     rows, K = 256, 128

@@ -8,8 +8,7 @@ import torch
 from oracle import moe, nvfp4
 from nvfp4_moe_grouped_token_b200 import ops, workloads
 
-from _parity import (check_bf16, check_f32, check_weights_exact, dequant_weights, gemm_bound,
-                     sf_rowmajor)
+from _parity import (check_bf16, check_f32, check_weights_exact, dequant_weights, gemm_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +58,7 @@ class Problem:
         tok = self.tok[rows]
         q = self.q.cpu().numpy()
         assert np.array_equal(q[pr], self.qx["q"][tok])
-        sf = sf_rowmajor(self.sf, self.cap, self.K)
+        sf = ops.sf_kstep_to_rowmajor(self.sf.cpu(), self.cap, self.K).numpy()
         assert np.array_equal(sf[pr], self.qx["sf"][tok])
         sd = self.sdec.cpu().numpy()
         want = self.qx["s_dec"][tok] if self.per_token else np.full(len(rows), self.qx["s_dec"][0])

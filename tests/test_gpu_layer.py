@@ -8,7 +8,7 @@ import torch
 from oracle import moe, nvfp4
 from nvfp4_moe_grouped_token_b200 import ops, workloads
 
-from _parity import (check_bf16, check_weights_exact, dequant_weights, gemm_bound, sf_rowmajor,
+from _parity import (check_bf16, check_weights_exact, dequant_weights, gemm_bound,
                      swiglu_bound)
 
 pytestmark = pytest.mark.gpu
@@ -65,7 +65,7 @@ class Layer:
         # 3. x quantized once per token, scattered (exact)
         qx = nvfp4.quantize(x, self.per_token)
         xq = v["x_q"].cpu().numpy()
-        xsf = sf_rowmajor(v["x_sf"], cap, H)
+        xsf = ops.sf_kstep_to_rowmajor(v["x_sf"].cpu(), cap, H).numpy()
         assert np.array_equal(xq[pr], qx["q"][tok[rows]])
         assert np.array_equal(xsf[pr], qx["sf"][tok[rows]])
         sd_want = qx["s_dec"][tok[rows]] if self.per_token else np.full(len(rows), qx["s_dec"][0])
@@ -95,7 +95,7 @@ class Layer:
             amax = np.abs(valid_h).max()
             qh = nvfp4.quantize(h_gpu, False, amax_in=np.array([amax], np.float32))
         hq = v["h_q"].cpu().numpy()
-        hsf = sf_rowmajor(v["h_sf"], cap, I)
+        hsf = ops.sf_kstep_to_rowmajor(v["h_sf"].cpu(), cap, I).numpy()
         assert np.array_equal(hq[pr], qh["q"])
         assert np.array_equal(hsf[pr], qh["sf"])
         hsd = v["h_sdec"].cpu().numpy()[pr]
