@@ -45,8 +45,10 @@ def parse():
     ap.add_argument("--config", default="moe30b")
     ap.add_argument("--per-tensor", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-experts", type=int, default=6,
-                    help="experts whose routed rows form the CPU oracle sample")
+    ap.add_argument("--cpu-experts", type=int, default=30,
+                    help="experts whose routed rows form the cpu_baseline sample (~10 s of oracle work)")
+    ap.add_argument("--ref-experts", type=int, default=6,
+                    help="experts whose routed rows form each step of --impl reference (~2 s per step)")
     return ap.parse_args()
 
 
@@ -376,14 +378,14 @@ def run_reference(args, rank, world):
     inp = workloads.layer_inputs(cfg)
     wq = None
     for _ in range(args.warmup):
-        _, _, wq = oracle_sample(cfg, inp, args.cpu_experts, per_token, wq)
+        _, _, wq = oracle_sample(cfg, inp, args.ref_experts, per_token, wq)
     secs, rows = 0.0, 0
     for _ in range(args.steps):
-        s, r, wq = oracle_sample(cfg, inp, args.cpu_experts, per_token, wq)
+        s, r, wq = oracle_sample(cfg, inp, args.ref_experts, per_token, wq)
         secs += s
         rows += r
     value = rows / cfg.k / secs
-    sample = (f"routed rows of experts 0..{args.cpu_experts - 1} per step ({rows // args.steps} rows), "
+    sample = (f"routed rows of experts 0..{args.ref_experts - 1} per step ({rows // args.steps} rows), "
               f"rate per token = rows/s / k")
     return {
         "impl": "reference",
