@@ -152,6 +152,17 @@ def test_moe30b_layer_sampled():
     L.check(sample_tokens=np.arange(0, cfg.T, 509), check_weights=False)
 
 
+def test_moe30b_skew_layer_sampled():
+    """65536 tokens with Zipf-skewed routing (several empty experts, a few
+    experts above 5 % of the rows), per-token scaling as in the bench."""
+    cfg = workloads.CONFIGS["moe30b_skew"]
+    L = Layer(cfg, ops.SCALE_PER_TOKEN)
+    L.run()
+    counts = np.diff(L.v["offsets"].cpu().numpy())
+    assert (counts == 0).sum() >= 5 and counts.max() > 0.05 * cfg.T * cfg.k
+    L.check(sample_tokens=np.arange(0, cfg.T, 1021), check_weights=False)
+
+
 def test_dense4b_layer_sampled():
     cfg = workloads.CONFIGS["dense4b"]
     L = Layer(cfg, ops.SCALE_PER_TOKEN)
