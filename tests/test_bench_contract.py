@@ -1,0 +1,58 @@
+"""bench.py on the CPU: the reference arm's JSON line and the pure helpers
+that turn event times into the reported throughput and roofline figures."""
+import json
+import os
+import subprocess
+import sys
+
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from nvfp4_moe_grouped_token_b200 import workloads  # noqa: E402
+
+
+def test_layer_flops_closed_form():
+    cfg = workloads.CONFIGS["moe30b"]
+    f = bench.layer_flops(cfg)
+    # 2 * rows * K * N for each GEMM, rows = T * k = 131072
+    assert f["gate_up"] == 2 * 131072 * 2048 * 1536
+    assert f["down"] == 2 * 131072 * 768 * 2048
+    assert abs(f["total"] - 1.237e12) / 1.237e12 < 1e-3
+
+
+def test_stage_bytes_count_each_tensor_once():
+    cfg = workloads.CONFIGS["moe30b"]
+    b = bench.stage_bytes(cfg, 0)
+    R, H, I, E = 131072, 2048, 768, 128
+    nv = 0.5625
+    assert b["combine"] == R * H * 2 + 16384 * H * 2 + R * 8
+    assert b["down"] == R * I * nv + E * H * I * nv + R * H * 2
+    assert b["requant_h"] == R * I * (2 + nv)
+
+
+def test_job_throughput_is_all_tokens_over_slowest_rank():
+    assert bench.job_throughput(16384, 1, 1.0) == 16384e3
+    assert bench.job_throughput(16384, 4, 2.0) == 4 * 16384 / 2e-3
+
+
+def test_reference_arm_prints_one_contract_line():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
+                          "--ref-experts", "1"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["steps"] == 1 and d["warmup"] == 0 and d["n_gpus"] == 1
+    assert "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
