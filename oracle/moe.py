@@ -24,6 +24,11 @@ Readings taken where the pages are silent (also in the design doc):
        once to BF16; the requantize input is that BF16 h.
   R12  Down-projection rows are BF16; y[t] = BF16( sum_j w[t,j] * D[t,j] ) with
        the sum in fp64 in slot order.
+  R15  Top-k routing from FP32 router logits: the k experts with the largest
+       logits (softmax is monotone, so these are the k most probable; ties
+       go to the lower expert id), slots in descending logit order, and the
+       weights are the softmax renormalised over the chosen k (Qwen3-MoE
+       style), in fp64.
 """
 from __future__ import annotations
 
@@ -32,6 +37,29 @@ import numpy as np
 from . import nvfp4
 
 GROUP_ALIGN = 128
+
+
+def route_topk(logits: np.ndarray, k: int):
+    """R15: top-k experts per token from router logits [T][E] (FP32 values).
+
+    The choice is exact -- a comparison of the logits themselves, lower expert
+    id first on equal logits -- and the weights are
+    w_j = exp(l_j - l_max) / sum_{i in top-k} exp(l_i - l_max) in fp64.
+    Returns idx int32 [T][k] and w float64 [T][k]."""
+    logits = np.asarray(logits, dtype=np.float64)
+    T, E = logits.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    ids = np.arange(E)
+    for t in range(T):
+        # descending logit, ascending id on ties: lexsort sorts by its last key first
+        order = np.lexsort((ids, -logits[t]))[:k]
+        idx[t] = order
+        z = np.exp(logits[t, order] - logits[t, order[0]])
+        w[t] = z / z.sum()
+    return idx, w
 
 
 def permutation(topk_idx: np.ndarray, num_experts: int):
