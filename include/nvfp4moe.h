@@ -113,6 +113,25 @@ int nvfp4_quantize(const void *x, int64_t M, int64_t K, const float *amax_in,
                    float *amax_out, uint8_t *q, uint8_t *scales, float *s_dec,
                    uint32_t flags, nvfp4moe_stream_t stream);
 
+/* -------------------------------------------------------------- routing -- */
+/* Top-k routing from router logits, on the device: the inputs of
+ * moe_permute without a trip through the host.  The pages' MoE learner runs
+ * Qwen3-30B-A3B (news.hamidun.com "miniTE ... 1.39x": 128 experts, 8 active
+ * per token) and keeps the token-wise path's metadata on the device
+ * (www.aib.vote "miniTE report", paragraph 4); the routing rule itself is not
+ * on the pages and follows Qwen3-MoE: for each token the k experts with the
+ * largest logits (ties to the lower expert id), slots in descending logit
+ * order, weights = softmax over the chosen k.  The choice compares the FP32
+ * logits exactly; the weights are FP32 (expf, one IEEE division each).
+ *   logits    [T][E] FP32 router logits (the dense router GEMM's output,
+ *             computed by the caller), finite values
+ *   topk_idx  [T][k] int32 expert ids (out)
+ *   topk_w    [T][k] FP32 weights, summing to 1 per token (out)
+ * Requirements: 1 <= k <= min(E, 32), E <= 1024; T == 0 is a no-op.
+ * NVFP4MOE_ERR_UNSUPPORTED_SHAPE beyond those limits. */
+int moe_route_topk(const float *logits, int64_t T, int E, int k, int32_t *topk_idx,
+                   float *topk_w, nvfp4moe_stream_t stream);
+
 /* ------------------------------------------------------------- permute -- */
 /* Token-to-expert permutation into a contiguous per-expert layout with
  * device-side group offsets (www.aib.vote "miniTE report", paragraph 4:

@@ -1,0 +1,122 @@
+// Top-k routing from FP32 router logits, on the device.
+//
+// The MoE learner's layer (news.hamidun.com "miniTE ... Qwen3-30B-A3B":
+// 128 experts, 8 active per token) starts from each token's router logits.
+// The pages say the token-wise path keeps its metadata on the device
+// (www.aib.vote "miniTE report, NVFP4 RL stability", paragraph 4); this
+// kernel turns logits into the topk_idx / topk_w the permutation consumes, so
+// nothing about the routing goes through the host.  The rule (the pages give
+// none; Qwen3-MoE style): the k experts with the largest logits, ties to the
+// lower expert id, slots in descending order, weights = softmax renormalised
+// over the chosen k.  The choice compares the FP32 logits exactly, so it is
+// bit-reproducible; only the weights carry rounding (expf and one division).
+//
+// One warp per token: lane l holds logits l, l+32, ...; each of the k rounds
+// is a warp arg-best under the strict order (larger logit, then lower id),
+// so every lane agrees on the winner whatever the reduction order.
+#include <climits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4moe {
+
+namespace {
+
+constexpr int kRouteWarps = 8;
+
+// (va, ia) ranks before (vb, ib): larger logit first, then lower expert id
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+template <int NE>   // logits per lane: E <= 32 * NE
+__global__ void __launch_bounds__(kRouteWarps * 32)
+    k_route_topk(const float *__restrict__ logits, int64_t T, int E, int k, int32_t *__restrict__ idx_out,
+                 float *__restrict__ w_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float *row = logits + t * E;
+  float v[NE];
+  uint32_t taken = 0;   // bit i: expert i*32 + lane already chosen (or beyond E)
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int e = i * 32 + lane;
+    v[i] = e < E ? __ldg(row + e) : 0.0f;
+    if (e >= E) taken |= 1u << i;
+  }
+  int my_id = 0;        // slot `lane` for lane < k
+  float my_v = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bv = 0.0f;
+    int bi = INT_MAX;   // INT_MAX: this lane has nothing left
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      const int e = i * 32 + lane;
+      if (!((taken >> i) & 1u) && (bi == INT_MAX || ranks_before(v[i], e, bv, bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != INT_MAX && (bi == INT_MAX || ranks_before(ov, oi, bv, bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    // k <= E, so a winner exists; its owner marks it taken
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) {
+      my_id = bi;
+      my_v = bv;
+    }
+  }
+  // weights: exp(l_j - l_max) over the chosen, normalised; the sum is a fixed
+  // butterfly, so the result does not depend on anything but the logits
+  const float m = __shfl_sync(0xffffffffu, my_v, 0);
+  const float z = lane < k ? expf(my_v - m) : 0.0f;
+  float s = z;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane < k) {
+    idx_out[t * k + lane] = my_id;
+    w_out[t * k + lane] = __fdiv_rn(z, s);
+  }
+}
+
+template <int NE>
+cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int32_t *idx, float *w, cudaStream_t s) {
+  const int64_t blocks = (T + kRouteWarps - 1) / kRouteWarps;
+  k_route_topk<NE><<<(unsigned)blocks, kRouteWarps * 32, 0, s>>>(logits, T, E, k, idx, w);
+  return cudaGetLastError();
+}
+
+bool aligned16_ptr(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace nvfp4moe
+
+using namespace nvfp4moe;
+
+extern "C" int moe_route_topk(const float *logits, int64_t T, int E, int k, int32_t *topk_idx, float *topk_w,
+                              nvfp4moe_stream_t stream) {
+  if (T < 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32 || k > E) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return NVFP4MOE_OK;
+  if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16_ptr(logits) || !aligned16_ptr(topk_idx) || !aligned16_ptr(topk_w))
+    return NVFP4MOE_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (E <= 32) e = launch_topk<1>(logits, T, E, k, topk_idx, topk_w, s);
+  else if (E <= 64) e = launch_topk<2>(logits, T, E, k, topk_idx, topk_w, s);
+  else if (E <= 128) e = launch_topk<4>(logits, T, E, k, topk_idx, topk_w, s);
+  else if (E <= 256) e = launch_topk<8>(logits, T, E, k, topk_idx, topk_w, s);
+  else if (E <= 512) e = launch_topk<16>(logits, T, E, k, topk_idx, topk_w, s);
+  else e = launch_topk<32>(logits, T, E, k, topk_idx, topk_w, s);
+  return e == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
+}

@@ -46,6 +46,7 @@ _SIGS = {
     "moe_permute_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "moe_route_topk": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
     "moe_quantize_permute": (_i32, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _i64, _u32, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64,
@@ -143,6 +144,14 @@ def moe_permute(topk_idx, E, offsets, padded_offsets, perm, inv_perm, workspace,
     _check(lib().moe_permute(_p(topk_idx), T, k, E, _p(offsets), _p(padded_offsets), _p(perm),
                              _p(inv_perm), _p(workspace), workspace.numel() * workspace.element_size(),
                              _stream(stream)), "moe_permute")
+
+
+def moe_route_topk(logits, k, topk_idx, topk_w, stream=None):
+    """moe_route_topk: logits [T][E] FP32 -> topk_idx [T][k] int32, topk_w [T][k] FP32."""
+    _dev(logits, topk_idx, topk_w)
+    T, E = logits.shape
+    _check(lib().moe_route_topk(_p(logits), T, E, k, _p(topk_idx), _p(topk_w), _stream(stream)),
+           "moe_route_topk")
 
 
 def moe_permute_noalloc(topk_idx, E, offsets, padded_offsets, perm, inv_perm, stream=None):

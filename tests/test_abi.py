@@ -43,6 +43,18 @@ def test_permute_checks():
     assert L.moe_permute(P16, 8, 40, 4, P16, P16, P16, P16, P16, 1 << 20, None) == -1
 
 
+def test_route_topk_checks():
+    r = L.moe_route_topk
+    assert r(P16, 8, 4, 8, P16, P16, None) == -3             # k > E
+    assert r(P16, 8, 2000, 8, P16, P16, None) == -3          # E > 1024
+    assert r(P16, 8, 128, 40, P16, P16, None) == -3          # k > 32
+    assert r(P16, 8, 128, 0, P16, P16, None) == -1
+    assert r(P16, -1, 128, 8, P16, P16, None) == -1
+    assert r(P16, 0, 128, 8, None, None, None) == 0          # empty: no-op
+    assert r(None, 8, 128, 8, P16, P16, None) == -1
+    assert r(P_ODD, 8, 128, 8, P16, P16, None) == -2
+
+
 def test_permute_workspace_size_grows_with_tokens():
     a = ops.moe_permute_workspace_size(128, 8, 128)
     b = ops.moe_permute_workspace_size(129, 8, 128)

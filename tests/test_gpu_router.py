@@ -1,0 +1,98 @@
+"""Top-k routing from router logits on the GPU against the oracle's router
+(reading R15): expert ids bit-exact, weights within a tolerance derived from
+the FP32 arithmetic, and the routed result feeding the permutation."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe
+from nvfp4_moe_grouped_token_b200 import ops
+
+pytestmark = pytest.mark.gpu
+
+# Weight tolerance, relative: expf is within 2 ulp (2^-22); l_j - l_max is one
+# FP32 subtraction (|error| <= 2^-24 * 16 for the N(0,1)-sized logits used
+# here, about 1e-6 relative after exp); the sum over at most 32 slots is 5
+# butterfly roundings and the division one more: about 2e-6 in all, 4e-6 with
+# margin.
+W_RTOL = 4e-6
+
+
+def _logits(T, E, seed, ties=False):
+    g = torch.Generator().manual_seed(seed)
+    lg = torch.randn(T, E, generator=g, dtype=torch.float32)
+    if ties:   # many exact ties: values on a 0.25 grid
+        lg = torch.round(lg * 4) / 4
+    return lg
+
+
+def _route_gpu(lg, k):
+    T, E = lg.shape
+    idx = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda")
+    ops.moe_route_topk(lg.cuda(), k, idx, w)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), w.cpu().numpy()
+
+
+def _check(lg, k):
+    idx, w = _route_gpu(lg, k)
+    ref_idx, ref_w = moe.route_topk(lg.numpy(), k)
+    assert np.array_equal(idx, ref_idx)
+    err = np.abs(w.astype(np.float64) - ref_w)
+    assert np.all(err <= W_RTOL * ref_w + 1e-38), float((err / ref_w).max())
+
+
+@pytest.mark.parametrize("T,E,k", [(5000, 128, 8), (777, 16, 4), (300, 1, 1), (257, 33, 1),
+                                   (200, 1000, 32), (129, 64, 32), (64, 256, 8), (64, 512, 16)])
+def test_route_topk_matches_oracle(T, E, k):
+    _check(_logits(T, E, seed=E * 31 + k), k)
+
+
+def test_route_topk_ties_go_to_the_lower_id():
+    _check(_logits(2000, 128, seed=9, ties=True), 8)
+    idx, w = _route_gpu(torch.zeros(5, 128), 8)
+    assert np.array_equal(idx, np.tile(np.arange(8), (5, 1)))
+    assert np.allclose(w, 1 / 8, rtol=0, atol=1e-7)
+
+
+def test_route_topk_empty_is_noop():
+    idx = torch.full((0, 8), -7, dtype=torch.int32, device="cuda")
+    w = torch.zeros(0, 8, dtype=torch.float32, device="cuda")
+    ops.moe_route_topk(torch.zeros(0, 128, device="cuda"), 8, idx, w)
+    torch.cuda.synchronize()
+
+
+def test_routed_tokens_permute_like_the_oracle():
+    """Logits -> device top-k -> device permutation, against the oracle's
+    top-k and permutation of the same logits (16384 tokens, 128 experts, top-8)."""
+    T, E, k = 16384, 128, 8
+    lg = _logits(T, E, seed=11)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ops.moe_route_topk(lg.cuda(), k, idx, w)
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    pad = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(ops.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
+    ops.moe_permute(idx, E, off, pad, perm, inv, ws)
+    assert ops.device_status(ws) == 0
+    ref_idx, _ = moe.route_topk(lg.numpy(), k)
+    info = moe.permutation(ref_idx, E)
+    assert np.array_equal(off.cpu().numpy(), info["offsets"])
+    assert np.array_equal(perm.cpu().numpy(), info["perm"])
+    assert np.array_equal(inv.cpu().numpy(), info["inv_perm"])
+    # the routing kernel's time at this shape (reported, not asserted)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lgd = lg.cuda()
+    for _ in range(3):
+        ops.moe_route_topk(lgd, k, idx, w)
+    e0.record()
+    for _ in range(20):
+        ops.moe_route_topk(lgd, k, idx, w)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / 20 * 1e3
+    print(f"moe_route_topk T={T} E={E} k={k}: {us:.1f} us per call "
+          f"({T * E * 4 / (us * 1e-6) / 1e9:.0f} GB/s of logits)")
