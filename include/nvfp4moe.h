@@ -96,6 +96,14 @@ int nvfp4moe_version(void);
  * NVFP4MOE_ERR_DEVICE_TIMEOUT.  This is the one call that blocks the host. */
 int nvfp4moe_device_status(void *workspace, nvfp4moe_stream_t stream);
 
+/* Self-test of the failure path every kernel's waits share (no counterpart on
+ * the pages): enqueues one kernel that waits on a barrier nothing completes.
+ * After the wait bound (2 s) the kernel records a timeout in the error word
+ * of `workspace` (16 bytes at least) and returns; nothing faults and the
+ * context stays usable.  A following nvfp4moe_device_status() returns
+ * NVFP4MOE_ERR_DEVICE_TIMEOUT. */
+int nvfp4moe_wait_selftest(void *workspace, nvfp4moe_stream_t stream);
+
 /* ------------------------------------------------------------ quantize -- */
 /* NVFP4-quantize x [M][K] BF16 (row-major).  The token-wise NVFP4 path with
  * amax reuse (www.aib.vote "miniTE report", paragraph 4).

@@ -132,6 +132,13 @@ const char *nvfp4moe_status_string(int status) {
 
 int nvfp4moe_version(void) { return 100; }
 
+int nvfp4moe_wait_selftest(void *workspace, nvfp4moe_stream_t stream) {
+  if (workspace == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  NVFP4MOE_TRY(launch_wait_selftest(static_cast<int *>(workspace), st(stream)));
+  return NVFP4MOE_OK;
+}
+
 int nvfp4moe_device_status(void *workspace, nvfp4moe_stream_t stream) {
   if (workspace == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
   int words[2] = {0, 0};

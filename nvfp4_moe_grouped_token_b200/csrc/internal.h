@@ -112,6 +112,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const void *d, const int32_t *inv_perm, const float *w, int64_t T, int k,
                            int64_t H, void *y, cudaStream_t s);
 
+cudaError_t launch_wait_selftest(int *err, cudaStream_t s);
 cudaError_t launch_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies, int mode,
                              long long *cycles, int *err, const uint8_t *gsrc, int grid, cudaStream_t s);
 

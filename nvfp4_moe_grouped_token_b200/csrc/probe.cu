@@ -234,6 +234,27 @@ __global__ void __launch_bounds__(160, 1)
 
 }  // namespace
 
+// Self-test of the bounded wait: one thread waits for a phase of an mbarrier
+// that nothing arrives on, through the same routine every kernel of the
+// library waits with.  After the bound it records kDevTimeout (detail 990)
+// in the error word and the kernel returns; nothing faults or hangs.
+__global__ void k_wait_selftest(int *err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, err, 990);
+}
+
+cudaError_t launch_wait_selftest(int *err, cudaStream_t s) {
+  k_wait_selftest<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies, int mode,
                              long long *cycles, int *err, const uint8_t *gsrc, int grid, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k_mma_probe, cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);

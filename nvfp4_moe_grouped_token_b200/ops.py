@@ -42,6 +42,7 @@ _SIGS = {
     "nvfp4moe_status_string": (ctypes.c_char_p, [_i32]),
     "nvfp4moe_version": (_i32, []),
     "nvfp4moe_device_status": (_i32, [_vp, _vp]),
+    "nvfp4moe_wait_selftest": (_i32, [_vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _u32, _vp]),
     "moe_permute_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -125,6 +126,12 @@ def _dev(*ts):
 def device_status(workspace: torch.Tensor, stream=None) -> int:
     """nvfp4moe_device_status: synchronizes; returns and clears the error word."""
     return lib().nvfp4moe_device_status(_p(workspace), _stream(stream))
+
+
+def wait_selftest(workspace: torch.Tensor, stream=None):
+    """nvfp4moe_wait_selftest: a kernel whose bounded wait runs out (~2 s)."""
+    _dev(workspace)
+    _check(lib().nvfp4moe_wait_selftest(_p(workspace), _stream(stream)), "nvfp4moe_wait_selftest")
 
 
 def nvfp4_quantize(x, q, scales, s_dec, flags=0, amax_in=None, amax_out=None, stream=None):
