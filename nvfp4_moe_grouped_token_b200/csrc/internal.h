@@ -10,7 +10,7 @@ namespace nvfp4moe {
 enum QuantMode : int {
   kQuantPlain = 0,     // row i -> row i (nvfp4_quantize)
   kQuantScatter = 1,   // token t -> its k rows in the padded grouped layout
-  kQuantRequant = 2,   // padded row p of h -> row p (valid rows only)
+  kQuantRequant = 2,   // padded row p of h -> row p, amax given (k_requant_blocks)
   kQuantWeights = 3,   // expert e row n -> expert e row interleave(n)
 };
 
@@ -24,7 +24,7 @@ enum SfLayout : int { kSfRowMajor = 0, kSfMma = 1, kSfKStep = 2 };
 
 struct QuantParams {
   const void *x = nullptr;          // BF16 source
-  int64_t tasks = 0;                // rows (plain), tokens (scatter), T*k (requant), E*N (weights)
+  int64_t tasks = 0;                // rows (plain), tokens (scatter), E*N (weights); requant walks rows_cap
   int64_t K = 0;                    // elements per row
   int mode = kQuantPlain;
   // amax: amax_src is the per-tensor value (index 0), per-row values, or per

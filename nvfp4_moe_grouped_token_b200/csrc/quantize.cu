@@ -79,27 +79,12 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   const int64_t nblk = K >> 4;
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(p.x);
 
-  // ---- source row ----------------------------------------------------------
-  int64_t src_row = task;
+  // ---- source row (plain, scatter, weights: the task's own row) ------------
   int64_t my_dest = -1;          // lane j < ndest holds destination j
   int ndest = 1;
   int64_t amax_index = 0;
   int64_t expert = 0;
-  if (p.mode == kQuantRequant) {
-    const int32_t *off = p.offsets;
-    if (task >= (int64_t)__ldg(off + p.E)) return;
-    int lo = 0, hi = p.E;                      // off[lo] <= task < off[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if ((int64_t)__ldg(off + mid) <= task) lo = mid; else hi = mid;
-    }
-    const int64_t pr = task - __ldg(off + lo) + __ldg(p.padded_offsets + lo);
-    if (pr >= p.rows_cap) return;
-    src_row = pr;
-    my_dest = pr;
-    amax_index = p.amax_rows ? pr : 0;
-  }
-  const uint4 *src = reinterpret_cast<const uint4 *>(xb + src_row * K);
+  const uint4 *src = reinterpret_cast<const uint4 *>(xb + task * K);
 
   // ---- load the row (registers when it fits) before anything that waits ---
   uint4 cache[NB > 0 ? NB : 1][2];
@@ -117,8 +102,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
   }
 
   // ---- destination row(s), amax source ----------------------------------
-  if (p.mode == kQuantRequant) {
-  } else if (p.mode == kQuantPlain) {
+  if (p.mode == kQuantPlain) {
     my_dest = task;
     amax_index = p.amax_rows ? task : 0;
   } else if (p.mode == kQuantScatter) {
@@ -405,7 +389,10 @@ cudaError_t launch_amax(const void *x, int64_t seg_len, int64_t nseg, float *out
 
 cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
   if (p.tasks <= 0) return cudaSuccess;
-  if (p.mode == kQuantRequant && !p.compute_row_amax) {
+  if (p.mode == kQuantRequant) {
+    // h is requantized with the amax the GEMM epilogue reduced; there is no
+    // requantization that computes its own amax
+    if (p.compute_row_amax) return cudaErrorInvalidValue;
     const uint32_t nblk = (uint32_t)(p.K / 16);
     // every padded row below rows_cap, every block; 32-bit indices
     if (p.rows_cap * (int64_t)nblk >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
