@@ -39,7 +39,7 @@ FP4_PER_BF16 = 4.0        # nominal dense FP4 : BF16 tensor throughput (9 : 2.25
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="moe30b")
@@ -64,54 +64,103 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed loop runs."""
+    """SM clocks and clock-event (throttle) reasons of one GPU, sampled while
+    the timed loop runs: read-only NVML queries every 5 ms, else nvidia-smi
+    every 200 ms.  Samples between mark_begin() and mark_end() are the ones
+    reported."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
     def __init__(self, index: int):
         self.index = index
+        self.samples = []          # (host time, sm MHz, max sm MHz, set of active reasons)
+        self.t0 = self.t1 = None
+        self.source = None
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.stop_event = threading.Event()
+
+    def _nvml(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            props = torch.cuda.get_device_properties(self.index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (FileNotFoundError, OSError):
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=lambda: self.lines.extend(self.proc.stdout), daemon=True)
+            nv, h = self._nvml()
+
+            def loop():
+                while not self.stop_event.is_set():
+                    try:
+                        t = time.perf_counter()
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+                        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((t, sm, mx, {n for n, b in self.REASONS if bits & b}))
+                    except Exception:
+                        pass
+                    self.stop_event.wait(0.005)
+            self.source = "nvml"
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (FileNotFoundError, OSError):
+                self.proc = None
+                return
+
+            def loop():
+                names = [n for n, _ in self.REASONS]
+                for ln in self.proc.stdout:
+                    p = [x.strip() for x in ln.split(",")]
+                    if len(p) < 9:
+                        continue
+                    try:
+                        self.samples.append((time.perf_counter(), float(p[1]), float(p[2]),
+                                             {n for n, v in zip(names, p[5:9]) if v.lower() == "active"}))
+                    except ValueError:
+                        continue
+            self.source = "nvidia-smi"
+        self.thread = threading.Thread(target=loop, daemon=True)
         self.thread.start()
 
+    def mark_begin(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            p = [x.strip() for x in ln.split(",")]
-            if len(p) < 9:
-                continue
+        self.stop_event.set()
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(p[1]))
-                mx.append(float(p[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, p[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml and nvidia-smi unavailable"]}
+        inside = [x for x in self.samples
+                  if self.t0 is not None and self.t1 is not None and self.t0 <= x[0] <= self.t1]
+        use = inside if inside else self.samples[-3:]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": self.source}
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": max(x[2] for x in use),
+                "reasons": sorted(set().union(*(x[3] for x in use))), "samples": len(use),
+                "in_timed_region": bool(inside), "source": self.source}
 
 
 def layer_flops(cfg) -> dict:
@@ -199,14 +248,16 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
-    time.sleep(0.4)
+    time.sleep(0.2)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    clocks.mark_begin()
     t_start.record(stream)
     for i in range(args.steps):
         ops.moe_expert_layer_profiled(x, idx, w, wgu, wdn, y, ws, evs[i], flags)
     t_end.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()

@@ -56,3 +56,41 @@ def test_reference_arm_prints_one_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_clock_sampler_reports_the_timed_window_from_nvml(monkeypatch):
+    """A fake NVML: idle clocks before the window, loaded clocks with the power
+    cap active inside it, thermal slowdown after it."""
+    import time
+    import types
+
+    phase = {"p": "before"}
+    fake = types.ModuleType("pynvml")
+    fake.NVML_CLOCK_SM = 0
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByIndex = lambda i: ("gpu", i)
+
+    def by_bus(_):
+        raise RuntimeError("no such bus id")
+    fake.nvmlDeviceGetHandleByPciBusId = by_bus
+    fake.nvmlDeviceGetClockInfo = lambda h, kind: {"before": 300, "in": 1900, "after": 1100}[phase["p"]]
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: {"before": 0x1, "in": 0x4, "after": 0x40}[phase["p"]]
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.05)
+    phase["p"] = "in"
+    time.sleep(0.02)
+    c.mark_begin()
+    time.sleep(0.08)
+    c.mark_end()
+    time.sleep(0.02)
+    phase["p"] = "after"
+    time.sleep(0.05)
+    r = c.stop()
+    assert r["source"] == "nvml" and r["in_timed_region"] is True
+    assert r["samples"] >= 3
+    assert r["sm_mhz"] == 1900 and r["sm_max_mhz"] == 1965
+    assert r["reasons"] == ["sw_power_cap"]
