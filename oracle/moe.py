@@ -13,7 +13,7 @@ Source passages
     policy, log-prob gap about 1e-8): results must not depend on how tokens are
     batched, which is why strict mode uses per-token scales.
 
-Readings taken where the pages are silent (also in the design doc):
+Readings taken where the pages are silent:
   R8   Rows are ordered by (expert, token, slot); each expert's group starts at
        a multiple of 128 rows in the padded layout.
   R9   GEMM: out[r, n] = sum_k x_hat_a[r, k] * x_hat_w[e(r), n, k] in fp64,

@@ -10,7 +10,7 @@ Source passages
     unsigned E4M3 (UE4M3) scale per 16 consecutive elements along K, and one
     FP32 global scale.
 
-Readings taken where the pages are silent (each is also listed in the design doc):
+Readings taken where the pages are silent:
   R1  E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; bit 3 is the sign.
   R2  UE4M3 = E4M3 with the sign bit 0: bias 7, 3 mantissa bits, subnormals
       m * 2^-9, largest finite 448; code 0x7F (NaN) is never produced.
