@@ -258,7 +258,8 @@ int moe_combine(const void *d, const int32_t *inv_perm, const float *topk_w,
  *   a fused SwiGLU epilogue that also reduces the amax of h  -> requantize h
  *   reusing that amax  -> down grouped GEMM  -> weighted combine.
  *   x         [T][H] BF16 activations
- *   topk_idx  [T][k] int32, topk_w [T][k] FP32 routing (router output)
+ *   topk_idx  [T][k] int32, topk_w [T][k] FP32 routing (router output, e.g.
+ *             moe_route_topk)
  *   w_gate_up prepared with NVFP4MOE_W_GATE_UP: E x [2I][H]
  *   w_down    prepared plainly: E x [H][I]
  *   y         [T][H] BF16 (out)
@@ -266,14 +267,14 @@ int moe_combine(const void *d, const int32_t *inv_perm, const float *topk_w,
  *   workspace moe_expert_layer_workspace_size() bytes; its named regions
  *             (offsets, perm, h, ...) are laid out by
  *             moe_expert_layer_workspace_offsets() for inspection.
- * Requirements: H % 256 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32. */
+ * Requirements: H % 256 == 0, I % 256 == 0, 1 <= E <= 1024, 1 <= k <= 32. */
 size_t moe_expert_layer_workspace_size(int64_t T, int64_t H, int64_t I, int E,
                                        int k, uint32_t flags);
 
 /* Byte offsets of the regions inside the layer workspace, in this order:
  * [0] error word, [1] offsets, [2] padded_offsets, [3] perm, [4] inv_perm,
- * [5] x codes (padded rows), [6] x scales (MMA layout), [7] x row S_dec,
- * [8] h BF16 (padded rows), [9] h amax, [10] h codes, [11] h scales,
+ * [5] x codes (padded rows), [6] x scales (K-step-major layout), [7] x row S_dec,
+ * [8] h BF16 (padded rows), [9] h amax, [10] h codes, [11] h scales (K-step-major),
  * [12] h row S_dec, [13] D BF16 (compact rows), [14] rows_cap (a count, not an
  * offset), [15] total bytes.  `out` must hold 16 int64 (host memory). */
 int moe_expert_layer_workspace_offsets(int64_t T, int64_t H, int64_t I, int E,
