@@ -109,23 +109,49 @@ __global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams
       base += c;
     }
   }
-  // inclusive scans of totals and padded totals over experts
-  int32_t v = (tid < E && s == 0) ? total : 0;
-  int32_t vp = (tid < E && s == 0) ? ((total + 127) / 128) * 128 : 0;
-  scan_a[tid] = v;
-  scan_b[tid] = vp;
-  __syncthreads();
-  for (int o = 1; o < kScanThreads; o <<= 1) {
-    const int32_t a = tid >= o ? scan_a[tid - o] : 0;
-    const int32_t b = tid >= o ? scan_b[tid - o] : 0;
-    __syncthreads();
-    scan_a[tid] += a;
-    scan_b[tid] += b;
-    __syncthreads();
+  // inclusive scans of totals and padded totals over experts: a warp scan,
+  // then a scan of the 32 warp sums (two block barriers)
+  __shared__ int32_t wsum_a[kScanThreads / 32];
+  __shared__ int32_t wsum_b[kScanThreads / 32];
+  const int32_t v = (tid < E && s == 0) ? total : 0;
+  const int32_t vp = (tid < E && s == 0) ? ((total + 127) / 128) * 128 : 0;
+  const int lane = tid & 31, wid = tid >> 5;
+  int32_t ia = v, ib = vp;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t ya = __shfl_up_sync(0xffffffffu, ia, o);
+    const int32_t yb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += ya;
+      ib += yb;
+    }
   }
+  if (lane == 31) {
+    wsum_a[wid] = ia;
+    wsum_b[wid] = ib;
+  }
+  __syncthreads();
+  if (wid == 0) {                            // kScanThreads / 32 == 32 warp sums
+    const int32_t oa = wsum_a[lane], ob = wsum_b[lane];
+    int32_t xa = oa, xb = ob;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t ya = __shfl_up_sync(0xffffffffu, xa, o);
+      const int32_t yb = __shfl_up_sync(0xffffffffu, xb, o);
+      if (lane >= o) {
+        xa += ya;
+        xb += yb;
+      }
+    }
+    wsum_a[lane] = xa - oa;                  // sums of the warps before this one
+    wsum_b[lane] = xb - ob;
+  }
+  __syncthreads();
+  ia += wsum_a[wid];
+  ib += wsum_b[wid];
   if (tid < E) {
-    p.offsets[tid + 1] = scan_a[tid];
-    p.padded_offsets[tid + 1] = scan_b[tid];
+    p.offsets[tid + 1] = ia;
+    p.padded_offsets[tid + 1] = ib;
   }
   if (tid == 0) {
     p.offsets[0] = 0;
@@ -133,11 +159,10 @@ __global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams
   }
   if (p.zero_pad_rows != nullptr) {
     // a warp per group: its at most 127 padding rows in four 32-wide steps
+    scan_a[tid] = v;                         // count of group tid
+    scan_b[tid] = ib;                        // padded end of group tid
     __syncthreads();
-    if (tid < E) scan_a[tid] = v;            // counts again (the scan is done with scan_a)
-    __syncthreads();
-    const int lane = tid & 31;
-    for (int g = tid >> 5; g < E; g += kScanThreads / 32) {
+    for (int g = wid; g < E; g += kScanThreads / 32) {
       const int64_t end = scan_b[g];
       const int32_t cnt = scan_a[g];
       const int64_t start = end - (((int64_t)cnt + 127) / 128) * 128;
