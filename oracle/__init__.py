@@ -20,7 +20,9 @@ exactly as the quantizer on the GPU must do it; everything else (dequantize,
 GEMM, SwiGLU, combine) is fp64.
 
 Modules
-  nvfp4   -- E2M1 / UE4M3 codecs, BF16 rounding, quantize, dequantize
-  moe     -- permutation, grouped GEMM, SwiGLU + requantize, combine, the layer
+  nvfp4    -- E2M1 / UE4M3 codecs, BF16 rounding, quantize, dequantize
+  moe      -- routing, permutation, grouped GEMM, SwiGLU + requantize, combine,
+              the layer
+  backward -- the layer's gradients in the BF16-backward mode
 """
-from . import nvfp4, moe  # noqa: F401
+from . import nvfp4, moe, backward  # noqa: F401
