@@ -24,5 +24,6 @@ Modules
   moe      -- routing, permutation, grouped GEMM, SwiGLU + requantize, combine,
               the layer
   backward -- the layer's gradients in the BF16-backward mode
+  mxfp8    -- MXFP8 (E4M3 elements, E8M0 block scales) for the W4A8 variant
 """
-from . import nvfp4, moe, backward  # noqa: F401
+from . import nvfp4, moe, backward, mxfp8  # noqa: F401
