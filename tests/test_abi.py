@@ -120,3 +120,44 @@ def test_sf_layout_permutation_is_a_bijection():
     assert torch.equal(torch.sort(rm.reshape(-1)).values, flat)
     # one known position: row 37, block 5 -> atom 1 of m-tile 0, (37%32)*16 + (37//32)*4 + 1
     assert int(rm[37, 5]) == 1 * 512 + 5 * 16 + 1 * 4 + 1
+
+
+def test_quantize_permute_checks():
+    qp = L.moe_quantize_permute
+    a = [P16, P16, P16, P16]                       # topk_idx, inv_perm, offsets, padded_offsets
+    assert qp(P16, 8, 100, 2, 4, *a, None, P16, P16, P16, P16, 1024, 0, None) == -3    # K % 64
+    assert qp(P16, 8, 256, 40, 4, *a, None, P16, P16, P16, P16, 1024, 0, None) == -1   # k > 32
+    assert qp(P16, 0, 256, 2, 4, *a, None, P16, P16, P16, P16, 1024, 0, None) == 0     # empty: no-op
+    assert qp(None, 8, 256, 2, 4, *a, None, P16, P16, P16, P16, 1024, 0, None) == -1
+    assert qp(P_ODD, 8, 256, 2, 4, *a, None, P16, P16, P16, P16, 1024, 0, None) == -2
+    assert qp(P16, 8, 256, 2, 4, *a, None, None, P16, P16, P16, 1024, 0, None) == -1   # per tensor: amax needed
+
+
+def test_combine_checks():
+    c = L.moe_combine
+    assert c(P16, P16, P16, 8, 2, 100, P16, None) == -3       # H % 8
+    assert c(P16, P16, P16, 8, 0, 256, P16, None) == -1
+    assert c(P16, P16, P16, 0, 2, 256, P16, None) == 0        # empty: no-op
+    assert c(None, P16, P16, 8, 2, 256, P16, None) == -1
+    assert c(P_ODD, P16, P16, 8, 2, 256, P16, None) == -2
+
+
+def test_prepare_weights_checks():
+    pw = L.nvfp4_prepare_weights
+    out = ops._Weights(P16.value, P16.value, P16.value, P16.value, 0, 0, 0, 0)
+    assert pw(P16, 4, 256, 200, 0, ctypes.byref(out), None) == -3     # K % 256
+    assert pw(P16, 4, 300, 256, 0, ctypes.byref(out), None) == -3     # N % 256
+    assert pw(None, 4, 256, 256, 0, ctypes.byref(out), None) == -1
+    assert pw(P_ODD, 4, 256, 256, 0, ctypes.byref(out), None) == -2
+    bad = ops._Weights(None, P16.value, P16.value, P16.value, 0, 0, 0, 0)
+    assert pw(P16, 4, 256, 256, 0, ctypes.byref(bad), None) == -1
+
+
+def test_noalloc_and_diagnostic_checks():
+    na = L.moe_permute_noalloc
+    assert na(P16, 8, 2, 2000, P16, P16, P16, P16, None) == -3      # E > 1024
+    assert na(P16, 8, 40, 4, P16, P16, P16, P16, None) == -1        # k > 32
+    assert na(P16, 70000, 2, 4, P16, P16, P16, P16, None) == -6     # beyond the static scratch
+    assert L.nvfp4moe_wait_selftest(None, None) == -1
+    assert L.nvfp4moe_wait_selftest(P_ODD, None) == -2
+    assert L.nvfp4moe_device_status(None, None) == -1
