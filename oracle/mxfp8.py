@@ -1,5 +1,6 @@
-"""MXFP8 (E4M3 elements, E8M0 block scales) quantize / dequantize -- CPU
-oracle (test infrastructure only).
+"""MX formats for the W4A8 variant: MXFP8 activations (E4M3 elements) and
+MXFP4 weights (E2M1 elements), both with E8M0 block scales -- CPU oracle (test
+infrastructure only).
 
 Source passage: the miniTE pages' precision-mismatch study lists, next to the
 W4A4 NVFP4 path, variants with 8-bit activations in MXFP8 (W4A8) and 16-bit
@@ -15,6 +16,11 @@ Reading taken where the pages are silent:
        takes s = -127.  Each element is E4M3(V / X), round to nearest even,
        saturating at +-448 (V / X can reach 2^9 > 448); a negative value that
        rounds to zero keeps its sign (code 0x80).  E8M0 code = s + 127.
+  R18  MXFP4 weights for the same variant (the block-scaled MMA that takes
+       E4M3 activations takes E8M0 scales per 32 elements on both operands):
+       the same rule with E2M1 elements, s = floor(log2(amax_block)) - 2
+       (6 = 1.5 * 2^2), elements E2M1(V / X) round to nearest even,
+       saturating at +-6.
 """
 from __future__ import annotations
 
@@ -70,3 +76,30 @@ def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     s = scales.astype(np.int64) - 127
     v = e4m3_decode_signed(codes).reshape(M, K // BLOCK, BLOCK)
     return (v * np.ldexp(1.0, s)[:, :, None]).reshape(M, K)
+
+
+E2M1_EMAX = 2
+
+
+def quantize_mxfp4(w: np.ndarray):
+    """R18: w [N][K] (K % 32 == 0) -> E2M1 codes uint8 [N][K] (one per byte,
+    bit 3 the sign) and E8M0 scales uint8 [N][K/32]."""
+    w = np.asarray(w, dtype=np.float64)
+    N, K = w.shape
+    if K % BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    blocks = w.reshape(N, K // BLOCK, BLOCK)
+    amax = np.abs(blocks).max(axis=2)
+    _, p = np.frexp(amax)
+    s = np.clip(np.where(amax > 0, (p - 1) - E2M1_EMAX, -127), -127, 127).astype(np.int64)
+    v = blocks / np.ldexp(1.0, s)[:, :, None]
+    codes = nvfp4.e2m1_encode(v).reshape(N, K)
+    return codes, (s + 127).astype(np.uint8)
+
+
+def dequantize_mxfp4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    N, K = codes.shape
+    s = scales.astype(np.int64) - 127
+    v = nvfp4.e2m1_decode(codes).reshape(N, K // BLOCK, BLOCK)
+    return (v * np.ldexp(1.0, s)[:, :, None]).reshape(N, K)

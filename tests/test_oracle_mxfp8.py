@@ -70,3 +70,29 @@ def test_negative_values_that_round_to_zero_keep_the_sign():
     x[0, 1] = -2.0 ** -11                            # below half the smallest subnormal at s = 0
     codes, _ = mxfp8.quantize(x)
     assert codes[0, 1] == 0x80
+
+
+def test_mxfp4_scales_put_the_block_max_in_4_8_and_round_to_the_e2m1_grid():
+    w = _bf16((32, 256), 5, scale=0.02)
+    codes, sc = mxfp8.quantize_mxfp4(w)
+    s = sc.astype(np.int64) - 127
+    amax = np.abs(w.reshape(32, 8, 32)).max(axis=2)
+    ratio = amax / np.ldexp(1.0, s)
+    assert np.all((ratio >= 4) & (ratio < 8))
+    deq = mxfp8.dequantize_mxfp4(codes, sc)
+    # brute force: every element is the nearest point of the scaled E2M1 grid (saturating at 6)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    v = np.abs(w.reshape(32, 8, 32) / np.ldexp(1.0, s)[:, :, None]).reshape(-1)
+    got = np.abs(deq.reshape(32, 8, 32) / np.ldexp(1.0, s)[:, :, None]).reshape(-1)
+    dist = np.abs(v[:, None] - grid[None, :])
+    best = dist.min(axis=1)
+    assert np.all(np.abs(got - v) <= best + 1e-12)
+    assert np.all(got <= 6.0)
+
+
+def test_mxfp4_saturates_and_keeps_zero_blocks():
+    w = np.zeros((2, 32))
+    w[0, 0] = 7.5                                     # 4 <= 7.5 < 8 at s = 0 -> saturates to 6
+    codes, sc = mxfp8.quantize_mxfp4(w)
+    assert sc[0, 0] == 127 and mxfp8.dequantize_mxfp4(codes, sc)[0, 0] == 6.0
+    assert sc[1, 0] == 0 and not codes[1].any()
