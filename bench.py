@@ -468,10 +468,9 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if True:
-            res, cfg = run_ours(args, rank, world, local_rank)
-            if rank == 0 and world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_experts, not args.per_tensor)
+        res, cfg = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_experts, not args.per_tensor)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:
