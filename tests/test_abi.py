@@ -161,3 +161,35 @@ def test_noalloc_and_diagnostic_checks():
     assert L.nvfp4moe_wait_selftest(None, None) == -1
     assert L.nvfp4moe_wait_selftest(P_ODD, None) == -2
     assert L.nvfp4moe_device_status(None, None) == -1
+
+
+def test_header_compiles_as_c99_and_the_library_links_from_c(tmp_path):
+    """The boundary is plain C: a C99 program includes the header, links the
+    library and calls entry points that return before any launch."""
+    import os
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(ops.LIB_PATH)
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "nvfp4moe.h"
+int main(void) {
+  int bad_k = moe_combine((void *)0x100000, (const int32_t *)0x100000, (const float *)0x100000,
+                          8, 0, 256, (void *)0x100000, (nvfp4moe_stream_t)0);
+  size_t ws = moe_expert_layer_workspace_size(16384, 2048, 768, 128, 8, NVFP4MOE_SCALE_PER_TOKEN);
+  printf("%d %s %d %d\n", nvfp4moe_version() >= 100, nvfp4moe_status_string(NVFP4MOE_OK), bad_k, ws > 0);
+  return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"), str(src),
+                         "-o", str(exe), "-L", lib_dir, "-lnvfp4moe", "-Wl,-rpath," + lib_dir],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    assert run.stdout.split() == ["1", "ok", "-1", "1"]
