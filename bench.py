@@ -1,10 +1,13 @@
 """Benchmark of the NVFP4 W4A4 MoE expert layer (one JSON line on rank 0).
 
-Workload: the Qwen3-30B-A3B-shaped expert layer -- 16384 tokens, hidden 2048,
-128 experts, top-8 softmax routing, gate_up 2048 -> 2x768 with SwiGLU and
-NVFP4 requantization, down 768 -> 2048 -- on seeded synthetic BF16 data.  A
-step is one moe_expert_layer call (every kernel of the path).  Per-token
-scaling (the token-wise path) is the default; --per-tensor switches.
+Headline workload: the Qwen3-30B-A3B-shaped expert layer -- 16384 tokens,
+hidden 2048, 128 experts, top-8 softmax routing, gate_up 2048 -> 2x768 with
+SwiGLU and NVFP4 requantization, down 768 -> 2048 -- on seeded synthetic BF16
+data.  A step is one moe_expert_layer call (every kernel of the path).
+Per-token scaling (the token-wise path) is the default; --per-tensor switches.
+At one GPU the same line also carries the other synthetic workloads (toy,
+dense Qwen3-4B-shaped, the Zipf-skewed 65536-token MoE layer) under
+"workloads", each with its own throughput, roofline, e2e and CPU baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -45,10 +48,16 @@ def parse():
     ap.add_argument("--config", default="moe30b")
     ap.add_argument("--per-tensor", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-experts", type=int, default=30,
+    ap.add_argument("--cpu-experts", type=int, default=8,
                     help="experts whose routed rows form the cpu_baseline sample (~10 s of oracle work)")
-    ap.add_argument("--ref-experts", type=int, default=6,
+    ap.add_argument("--ref-experts", type=int, default=2,
                     help="experts whose routed rows form each step of --impl reference (~2 s per step)")
+    ap.add_argument("--workloads", default="toy,dense4b,moe30b_skew",
+                    help="extra workloads measured at one GPU and reported under 'workloads' ('' = none)")
+    ap.add_argument("--workload-steps", type=int, default=20)
+    ap.add_argument("--no-backward", action="store_true", help="skip timing the BF16 backward")
+    ap.add_argument("--no-fast-combine", action="store_true",
+                    help="skip measuring the non-strict (FP32-reduction) combine beside the headline")
     return ap.parse_args()
 
 
@@ -170,20 +179,27 @@ def layer_flops(cfg) -> dict:
     return {"gate_up": gu, "down": dn, "total": gu + dn}
 
 
-def stage_bytes(cfg, counts_pad_rows: int) -> dict:
-    """Algorithmic HBM bytes per stage (each tensor read or written once)."""
+def stage_bytes(cfg, per_tensor: bool = False, fused_requant: bool = False) -> dict:
+    """Algorithmic HBM bytes per stage (each tensor read or written once).
+
+    h leaves the gate_up GEMM in BF16 and a second pass requantizes it; with
+    the requantization fused into the GEMM (per-token scales only) the GEMM's
+    output is h's NVFP4 codes and scales and there is no requant stage."""
+    fused = fused_requant and not per_tensor
     T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
     R = T * k
     nv = 0.5 + 1.0 / 16                 # NVFP4 bytes per element (codes + UE4M3 scale)
     w_gu = E * 2 * I * H * nv
     w_dn = E * H * I * nv
-    return {
+    out = {
         "quantize_permute": T * H * 2 + R * H * nv + R * 8,
-        "gate_up_swiglu": R * H * nv + w_gu + R * I * 2,
-        "requant_h": R * I * 2 + R * I * nv,
+        "gate_up_swiglu": R * H * nv + w_gu + (R * I * nv if fused else R * I * 2),
         "down": R * I * nv + w_dn + R * H * 2,
         "combine": R * H * 2 + T * H * 2 + R * 8,
     }
+    if not fused:
+        out["requant_h"] = R * I * 2 + R * I * nv
+    return out
 
 
 # ------------------------------------------------------- multi-rank ----
@@ -210,35 +226,75 @@ def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
 
 # --------------------------------------------------------------- ours ----
 
-def run_ours(args, rank, world, local_rank):
+def fp4_peak(reps: int = 3) -> dict:
+    """The block-scaled FP4 MMA's measured throughput on this GPU (the GEMM's
+    instruction and tile shape, operands in shared memory), best of `reps`
+    launches, with and without the scale writes the GEMM's feeders issue."""
+    from nvfp4_moe_grouped_token_b200 import ops
+    pure = max(ops.mma_peak(4000, scale_writes=False)["tflops"] for _ in range(reps))
+    fed = max(ops.mma_peak(4000, scale_writes=True)["tflops"] for _ in range(reps))
+    return {"mma_only": pure, "with_scale_writes": fed}
+
+
+def kernel_rooflines(cfg, stage_ms: dict, per_tensor: bool, pk: dict, fp4: dict, traffic, fused_requant=False):
+    """Every stage of the step against its own bound: HBM stages against the
+    measured copy bandwidth, the GEMMs against the measured FP4 MMA peak (and
+    the down GEMM, whose BF16 output dominates its bytes, against HBM too)."""
+    fl = layer_flops(cfg)
+    sb = stage_bytes(cfg, per_tensor, fused_requant)
+    out = []
+    for name, ms in stage_ms.items():
+        if name not in sb and name != "route":
+            continue
+        sec = ms * 1e-3
+        row = {"stage": name, "ms": ms}
+        if name == "route":
+            row.update(bound="latency", note="histogram + scan of the routing metadata (~1 MB)")
+        elif name in ("gate_up_swiglu", "down"):
+            f = fl["gate_up" if name == "gate_up_swiglu" else "down"]
+            row.update(bound="tensor" if name == "gate_up_swiglu" else "hbm",
+                       tflops=f / sec / 1e12, frac_fp4_peak=f / sec / 1e12 / fp4["mma_only"],
+                       gbs=sb[name] / sec / 1e9, frac_hbm=sb[name] / sec / 1e9 / pk["hbm_gbs"],
+                       algorithmic_bytes=sb[name], flop=f)
+            if name == "gate_up_swiglu":
+                row["traffic"] = traffic
+        else:
+            row.update(bound="hbm", gbs=sb[name] / sec / 1e9, frac_hbm=sb[name] / sec / 1e9 / pk["hbm_gbs"],
+                       algorithmic_bytes=sb[name])
+        out.append(row)
+    return out
+
+
+FAST_COMBINE_FLAG = 0x80     # NVFP4MOE_FAST_COMBINE
+FUSED_REQUANT_FLAG = 0x100   # NVFP4MOE_FUSED_REQUANT
+
+
+def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=True, extra_flags=0):
+    """Time `steps` layer steps (inputs resident in HBM) and the same number of
+    end-to-end steps from pinned host buffers.  Returns the measurement dict."""
     from nvfp4_moe_grouped_token_b200 import ops
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    cfg = rank_config(workloads.CONFIGS[args.config], rank, world)
-    flags = 0 if args.per_tensor else ops.SCALE_PER_TOKEN
+    flags = (0 if args.per_tensor else ops.SCALE_PER_TOKEN) | extra_flags
     inp = workloads.layer_inputs(cfg)
     x = inp["x"].to(dev)
     idx = inp["topk_idx"].to(dev)
     w = inp["topk_w"].to(dev)
     wgu = ops.nvfp4_prepare_weights(inp["w_gate_up"].to(dev), gate_up=True)
     wdn = ops.nvfp4_prepare_weights(inp["w_down"].to(dev), gate_up=False)
+    del inp["w_gate_up"], inp["w_down"]
     ws = torch.empty(ops.moe_expert_layer_workspace_size(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, flags),
                      dtype=torch.uint8, device=dev)
     y = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
+    for _ in range(warmup):
         ops.moe_expert_layer(x, idx, w, wgu, wdn, y, ws, flags)
-
-    for _ in range(args.warmup):
-        step()
     torch.cuda.synchronize()
     assert ops.device_status(ws) == 0
 
     # ---- timed region: K steps, stage events on the launching stream -----
     nstage = len(ops.STAGES)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(steps)]
     for row in evs:                          # materialise the events before timing
         for e in row:
             e.record(stream)
@@ -246,29 +302,34 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    time.sleep(0.2)
+    clocks = ClockSampler(dev.index) if clocks_for_timed else None
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.2)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    clocks.mark_begin()
+    if clocks is not None:
+        clocks.mark_begin()
     t_start.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         ops.moe_expert_layer_profiled(x, idx, w, wgu, wdn, y, ws, evs[i], flags)
     t_end.record(stream)
     torch.cuda.synchronize()
-    clocks.mark_end()
+    if clocks is not None:
+        clocks.mark_end()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks is not None else None
     assert ops.device_status(ws) == 0
 
     total_ms = t_start.elapsed_time(t_end)
-    step_ms = [evs[i][0].elapsed_time(evs[i][nstage]) for i in range(args.steps)]
-    stage_ms = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+    step_ms = [evs[i][0].elapsed_time(evs[i][nstage]) for i in range(steps)]
+    stage_ms = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
                 for j, name in enumerate(ops.STAGES)}
-    ms = max_over_ranks(total_ms / args.steps, world, dev)
+    if flags & FUSED_REQUANT_FLAG:
+        stage_ms.pop("requant_h")              # fused into gate_up: an empty interval
+    ms = max_over_ranks(total_ms / steps, world, dev)
 
     # ---- end to end through the public API with host buffers ----------------
     xh = inp["x"].pin_memory()
@@ -288,7 +349,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(3, args.steps // 2)
+    n_e2e = max(3, steps // 2)
     e0.record(stream)
     for _ in range(n_e2e):
         e2e_step()
@@ -298,50 +359,166 @@ def run_ours(args, rank, world, local_rank):
 
     fl = layer_flops(cfg)
     pk = peaks()
-    fp4_peak_sustained = pk["bf16_tflops_sustained"] * FP4_PER_BF16
-    gu_ms = stage_ms["gate_up_swiglu"]
-    gu_tflops = fl["gate_up"] / (gu_ms * 1e-3) / 1e12
-    traffic = load_traffic("gate_up_swiglu")
-    sb = stage_bytes(cfg, 0)
+    traffic = load_traffic("gate_up_swiglu") if cfg.name == "moe30b" else None
+    kern = kernel_rooflines(cfg, stage_ms, args.per_tensor, pk, fp4, traffic, bool(flags & FUSED_REQUANT_FLAG))
+    gu = next(r for r in kern if r["stage"] == "gate_up_swiglu")
+    bf16x4 = pk["bf16_tflops"] * FP4_PER_BF16
+    launches_per_step = 7 + (1 if args.per_tensor else 0) - (1 if flags & FUSED_REQUANT_FLAG else 0)
+    return {
+        "value": job_throughput(cfg.T, world, ms),
+        "ms_per_step": ms,
+        "tflops": world * fl["total"] / (ms * 1e-3) / 1e12,
+        "stages_ms": stage_ms,
+        "step_ms_min_max": [min(step_ms), max(step_ms)],
+        "roofline": {"kernel": "k_grouped_gemm (gate_up + SwiGLU epilogue)",
+                     "bound": "tensor", "achieved": gu["tflops"], "peak": fp4["mma_only"], "unit": "TFLOP/s",
+                     "frac": gu["tflops"] / fp4["mma_only"], "traffic": traffic,
+                     "peak_note": "block-scaled FP4 MMA (M128 N256 K64) measured in this process, operands in "
+                                  "shared memory (nvfp4moe_mma_peak)",
+                     "peak_with_scale_writes": fp4["with_scale_writes"],
+                     "frac_vs_bf16_burst_x4": gu["tflops"] / bf16x4,
+                     "bf16_burst_x4": bf16x4, "bf16_source": pk["source"],
+                     "frac_vs_nominal_9pf": gu["tflops"] / 9000.0,
+                     "kernels": kern},
+        "e2e": {"value": job_throughput(cfg.T, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4,
+                "d2h_bytes_per_step": yh.numel() * 2},
+        "gpu_launches": steps * launches_per_step,
+        "launches_per_step": launches_per_step,
+        "clocks": clk,
+    }
+
+
+def backward_flops(cfg) -> dict:
+    """The BF16 backward's products (2 * rows * K * N each): the recomputed
+    gate_up, dgrad of down, dgrad of gate_up, and the two weight gradients."""
+    R = cfg.T * cfg.k
+    H, I = cfg.H, cfg.I
+    f = {"gate_up_recompute": 2.0 * R * H * 2 * I, "dgrad_down": 2.0 * R * H * I, "dgrad_gate_up": 2.0 * R * 2 * I * H,
+         "wgrad_down": 2.0 * R * H * I, "wgrad_gate_up": 2.0 * R * 2 * I * H}
+    f["total"] = sum(f.values())
+    return f
+
+
+def measure_backward(cfg, dev, steps, warmup):
+    """Time moe_expert_layer_backward (BF16 backward of the layer, FP32 weight
+    gradients) on the workload, inputs resident in HBM."""
+    from nvfp4_moe_grouped_token_b200 import ops
+
+    inp = workloads.layer_inputs(cfg)
+    x, idx, w = inp["x"].to(dev), inp["topk_idx"].to(dev), inp["topk_w"].to(dev)
+    wgu, wdn = inp["w_gate_up"].to(dev), inp["w_down"].to(dev)
+    g = torch.Generator().manual_seed(77)
+    dy = torch.randn(cfg.T, cfg.H, generator=g).to(torch.bfloat16).to(dev)
+    ws = torch.empty(ops.moe_expert_layer_backward_workspace_size(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k), dtype=torch.uint8,
+                     device=dev)
+    dx = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    dtw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
+    dwgu = torch.empty(cfg.E, 2 * cfg.I, cfg.H, dtype=torch.bfloat16, device=dev)
+    dwdn = torch.empty(cfg.E, cfg.H, cfg.I, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        ops.moe_expert_layer_backward(x, idx, w, wgu, wdn, dy, dx, dtw, ws, dw_gate_up_bf16=dwgu, dw_down_bf16=dwdn)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ops.device_status(ws) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert ops.device_status(ws) == 0
+    ms = e0.elapsed_time(e1) / steps
+    fl = backward_flops(cfg)
+    pk = peaks()
+    tf = fl["total"] / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "tokens_per_s": cfg.T / (ms * 1e-3), "tflops": tf, "flop": fl["total"],
+            "frac_bf16_burst": tf / pk["bf16_tflops"], "bf16_peak": pk["bf16_tflops"], "bf16_source": pk["source"],
+            "weight_grads": "bf16", "steps": steps,
+            "note": "BF16-backward mode: exact gradient of the unquantized layer on BF16 operands (gate_up recomputed)"}
+
+
+WORKLOAD_NAMES = {
+    "toy": "toy NVFP4 MoE layer (E=4, T=256, top-2, K=256 -> N=512)",
+    "dense4b": "dense Qwen3-4B-shaped W4A4 MLP (T=8192, 2560 -> 2x9728 -> 2560, 0.1% outlier channels x30)",
+    "moe30b": "Qwen3-30B-A3B-shaped MoE expert layer (moe30b)",
+    "moe30b_skew": "Qwen3-30B-A3B-shaped MoE layer, 65536 tokens, Zipf(1.2) skewed routing (moe30b_skew)",
+}
+
+
+def run_ours(args, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = rank_config(workloads.CONFIGS[args.config], rank, world)
+    fp4 = fp4_peak()
+    m = measure_layer(cfg, args, world, dev, args.steps, args.warmup, fp4)
     result = {
         "metric": METRIC,
-        "value": job_throughput(cfg.T, world, ms),
+        "value": m["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms,
+        "ms_per_step": m["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 scales) -> f32 accumulate, bf16 out",
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, softmax top-8 routing)",
-        "config": {"workload": f"Qwen3-30B-A3B-shaped MoE expert layer ({cfg.name})", "tokens_per_gpu": cfg.T,
+        "config": {"workload": WORKLOAD_NAMES.get(cfg.name.split("+")[0], cfg.name), "tokens_per_gpu": cfg.T,
                    "hidden": cfg.H, "intermediate": cfg.I, "experts": cfg.E, "top_k": cfg.k,
                    "scaling_mode": "per-tensor" if args.per_tensor else "per-token",
                    "parallelism": f"dp{world} (replicas, no data-path collective)",
                    "l2": "no flush: per-step working set ~1.5 GB (weights 340 MB + activations) > 126 MB L2"},
-        "tflops": world * fl["total"] / (ms * 1e-3) / 1e12,
-        "stages_ms": stage_ms,
-        "step_ms_min_max": [min(step_ms), max(step_ms)],
-        "gemm": {"gate_up_tflops": gu_tflops,
-                 "down_tflops": fl["down"] / (stage_ms["down"] * 1e-3) / 1e12,
-                 "fp4_peak_tflops_sustained": fp4_peak_sustained,
-                 "down_hbm_gbs": sb["down"] / (stage_ms["down"] * 1e-3) / 1e9},
-        "quantizer_gbs": sb["quantize_permute"] / (stage_ms["quantize_permute"] * 1e-3) / 1e9,
-        "requant_gbs": sb["requant_h"] / (stage_ms["requant_h"] * 1e-3) / 1e9,
-        "combine_gbs": sb["combine"] / (stage_ms["combine"] * 1e-3) / 1e9,
-        "roofline": {"kernel": "k_grouped_gemm (gate_up + SwiGLU epilogue)", "bound": "tensor",
-                     "achieved": gu_tflops, "peak": fp4_peak_sustained, "unit": "TFLOP/s",
-                     "frac": gu_tflops / fp4_peak_sustained,
-                     "peak_note": f"{pk['source']} sustained bf16 x {FP4_PER_BF16:g} (nominal FP4:BF16 ratio)",
-                     "traffic": traffic},
-        "e2e": {"value": job_throughput(cfg.T, world, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4,
-                "d2h_bytes_per_step": yh.numel() * 2},
-        "gpu_launches": args.steps * (7 + (1 if args.per_tensor else 0)),
-        "clocks": clk,
+        "tflops": m["tflops"],
+        "stages_ms": m["stages_ms"],
+        "step_ms_min_max": m["step_ms_min_max"],
+        "quantizer_gbs": next(r["gbs"] for r in m["roofline"]["kernels"] if r["stage"] == "quantize_permute"),
+        "roofline": m["roofline"],
+        "e2e": m["e2e"],
+        "gpu_launches": m["gpu_launches"],
+        "clocks": m["clocks"],
+        "fp4_mma_peak_tflops": fp4,
     }
+    if world == 1 and not args.per_tensor and not args.no_fast_combine:
+        # the non-strict combine (FP32 reductions from the down GEMM's epilogue,
+        # no D round trip): measured beside the headline strict-order step
+        fc = measure_layer(cfg, args, world, dev, max(10, args.steps // 2), max(3, args.warmup), fp4,
+                           clocks_for_timed=False, extra_flags=FAST_COMBINE_FLAG)
+        result["fast_combine"] = {"value": fc["value"], "ms_per_step": fc["ms_per_step"],
+                                  "stages_ms": fc["stages_ms"],
+                                  "note": "NVFP4MOE_FAST_COMBINE: non-strict (reduction order varies), "
+                                          "not bitwise reproducible; the headline value is the strict-order path"}
+    if world == 1 and not args.per_tensor and not args.no_fast_combine:
+        # the requantization fused into the gate_up GEMM (opt-in): measured
+        # beside the headline's separate pass
+        fr = measure_layer(cfg, args, world, dev, max(10, args.steps // 2), max(3, args.warmup), fp4,
+                           clocks_for_timed=False, extra_flags=FUSED_REQUANT_FLAG)
+        result["fused_requant"] = {"value": fr["value"], "ms_per_step": fr["ms_per_step"],
+                                   "stages_ms": fr["stages_ms"],
+                                   "note": "NVFP4MOE_FUSED_REQUANT: requantization inside the gate_up GEMM "
+                                           "(bitwise the same outputs); off by default because it is slower"}
+    if world == 1 and not args.no_backward:
+        result["backward"] = measure_backward(cfg, dev, max(5, args.steps // 5), 2)
+        torch.cuda.empty_cache()
+    if world == 1 and args.workloads:
+        extra = {}
+        for name in [w for w in args.workloads.split(",") if w and w != args.config]:
+            wcfg = workloads.CONFIGS[name]
+            wm = measure_layer(wcfg, args, world, dev, args.workload_steps, max(3, args.warmup), fp4,
+                               clocks_for_timed=False)
+            extra[name] = {"workload": WORKLOAD_NAMES.get(name, name), "value": wm["value"], "unit": "tokens/s",
+                           "ms_per_step": wm["ms_per_step"], "tflops": wm["tflops"], "steps": args.workload_steps,
+                           "stages_ms": wm["stages_ms"], "roofline": wm["roofline"], "e2e": wm["e2e"],
+                           "gpu_launches": wm["gpu_launches"],
+                           "config": {"tokens": wcfg.T, "hidden": wcfg.H, "intermediate": wcfg.I,
+                                      "experts": wcfg.E, "top_k": wcfg.k, "routing": wcfg.routing}}
+            result["gpu_launches"] += wm["gpu_launches"]
+            torch.cuda.empty_cache()
+        result["workloads"] = extra
     return result, cfg
 
 
@@ -369,56 +546,62 @@ def load_traffic(kernel_key: str):
 # ------------------------------------------------------- oracle (CPU) ----
 
 def oracle_sample(cfg, inp, n_experts: int, per_token: bool, wq=None):
-    """Time the CPU oracle on the routed rows of the first n_experts experts
-    (a bounded slice of the same workload).  Returns (seconds, rows, weights)."""
+    """Time the C++ CPU oracle on the routed rows of the first n_experts
+    experts (a bounded slice of the same workload): quantize the tokens,
+    permute, gate_up GEMM, SwiGLU, BF16, requantize h, down GEMM, BF16 D.
+    The weights are quantized once, outside the timed part.  Returns
+    (seconds, rows, weights)."""
     import numpy as np
-    from oracle import moe, nvfp4
+    from oracle import cpp
 
     idx = inp["topk_idx"].numpy()
     if wq is None:
-        wgu = inp["w_gate_up"][:n_experts].float().numpy()
-        wdn = inp["w_down"][:n_experts].float().numpy()
-        wq = (moe.QuantWeights(wgu), moe.QuantWeights(wdn))
-        for e in range(n_experts):
-            wq[0].dequant(e), wq[1].dequant(e)
+        def deq(w):
+            out = np.empty(w.shape, np.float64)
+            for e in range(w.shape[0]):
+                q = cpp.quantize(w[e], False)
+                out[e] = cpp.dequantize(q["q"], q["sf"], q["s_dec"])
+            return out
+        wq = (deq(inp["w_gate_up"][:n_experts].float().numpy()), deq(inp["w_down"][:n_experts].float().numpy()))
     x = inp["x"].float().numpy()
     t0 = time.perf_counter()
-    info = moe.permutation(idx, cfg.E)
+    info = cpp.permutation(idx, cfg.E)
     hi = int(info["offsets"][n_experts])
-    rows = np.arange(hi)
-    tok = info["perm"][rows] // cfg.k
+    tok = info["perm"][:hi] // cfg.k
     utok = np.unique(tok)
-    qx = nvfp4.quantize(x[utok], per_token) if per_token else nvfp4.quantize(x, False)
-    xh_rows = nvfp4.dequantize(qx["q"], qx["sf"], qx["s_dec"])
     if per_token:
-        a = xh_rows[np.searchsorted(utok, tok)]
+        qx = cpp.quantize(x[utok], True)
+        a = cpp.dequantize(qx["q"], qx["sf"], qx["s_dec"])[np.searchsorted(utok, tok)]
     else:
-        a = xh_rows[tok]
+        qx = cpp.quantize(x, False)
+        a = cpp.dequantize(qx["q"], qx["sf"], qx["s_dec"])[tok]
     off = info["offsets"][: n_experts + 1]
-    gu = moe.grouped_gemm(a, off, wq[0].dequant)
-    h = nvfp4.round_to_bf16(moe.swiglu(gu, cfg.I))
-    qh = nvfp4.quantize(h, per_token)
-    hh = nvfp4.dequantize(qh["q"], qh["sf"], qh["s_dec"])
-    d = nvfp4.round_to_bf16(moe.grouped_gemm(hh, off, wq[1].dequant))
+    gu = cpp.grouped_gemm(a, off, wq[0])
+    h = cpp.round_to_bf16(cpp.swiglu(gu, cfg.I))
+    qh = cpp.quantize(h, per_token)
+    hh = cpp.dequantize(qh["q"], qh["sf"], qh["s_dec"])
+    d = cpp.round_to_bf16(cpp.grouped_gemm(hh, off, wq[1]))
     _ = d.sum()
     return time.perf_counter() - t0, hi, wq
 
 
 def cpu_cores_used():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else os.cpu_count()
-    except Exception:
-        return os.cpu_count()
+    """Threads the C++ oracle runs its GEMMs on (one per host core)."""
+    from oracle import cpp
+    return cpp.threads()
 
 
 def cpu_baseline(cfg, n_experts: int, per_token: bool):
     inp = workloads.layer_inputs(cfg)
+    n_experts = min(n_experts, cfg.E)
     secs, rows, _ = oracle_sample(cfg, inp, n_experts, per_token)
     return {"value": rows / cfg.k / secs, "unit": "tokens/s", "cores": cpu_cores_used(), "kind": "oracle",
             "sample": f"routed rows of experts 0..{n_experts - 1} ({rows} of {cfg.T * cfg.k} rows), "
                       f"rate reported per token = rows/s / k; {secs:.1f} s of CPU time"}
+
+
+# experts whose routed rows form each extra workload's cpu_baseline sample
+WORKLOAD_CPU_EXPERTS = {"toy": 4, "dense4b": 1, "moe30b_skew": 2}
 
 
 def run_reference(args, rank, world):
@@ -442,7 +625,7 @@ def run_reference(args, rank, world):
         "impl": "reference",
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (C++ oracle)", "data": "synthetic",
         "config": {"workload": f"Qwen3-30B-A3B-shaped MoE expert layer ({cfg.name})",
                    "tokens_per_gpu": cfg.T, "hidden": cfg.H, "intermediate": cfg.I, "experts": cfg.E,
                    "top_k": cfg.k, "scaling_mode": "per-tensor" if args.per_tensor else "per-token"},
@@ -471,6 +654,10 @@ def main():
         res, cfg = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_experts, not args.per_tensor)
+            for name, wl in res.get("workloads", {}).items():
+                # a smaller sample per extra workload (a few seconds each)
+                wl["cpu_baseline"] = cpu_baseline(workloads.CONFIGS[name], WORKLOAD_CPU_EXPERTS.get(name, 8),
+                                                  not args.per_tensor)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:

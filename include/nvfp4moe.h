@@ -86,6 +86,27 @@ typedef enum {
  * 0..I-1, up rows I..2I-1); store rows in the order the fused SwiGLU epilogue
  * reads (per 256-row tile: 128 gate rows then the matching 128 up rows). */
 #define NVFP4MOE_W_GATE_UP 0x10u
+/* moe_expert_layer with per-token scales: requantize h inside the gate_up
+ * GEMM launch instead of a separate pass.  The GEMM then walks each CTA's
+ * m-tiles with all their n-tiles in a row, so a row of h and its amax are
+ * complete inside one CTA, and two worker warps per CTA requantize an m-tile
+ * from L2 while the tensor cores run the next one.  Outputs are bitwise the
+ * same as the separate pass.  Measured on the Qwen3-30B-A3B-shaped layer it
+ * is slower than the separate pass (the requantization needs more warps than
+ * a GEMM CTA can give it), so it is off by default. */
+#define NVFP4MOE_FUSED_REQUANT 0x100u
+/* With NVFP4MOE_FUSED_REQUANT: keep h (BF16) readable in the workspace.
+ * Without it the fused path drops h's cache lines once requantized, without
+ * writing them to HBM, and the workspace's h region holds undefined values
+ * afterwards.  Outputs are identical either way. */
+#define NVFP4MOE_KEEP_H 0x20u
+/* moe_expert_layer, non-strict: the down GEMM's epilogue adds w[t][j] * D
+ * (FP32, before any BF16 rounding) straight into an FP32 accumulator of y
+ * with reductions (red.global.add), and a last pass rounds it to BF16, so D
+ * never goes to memory.  The order of the additions follows the GEMM's tile
+ * completion, so y is not bitwise reproducible: not allowed with
+ * NVFP4MOE_STRICT (NVFP4MOE_ERR_INVALID_ARG). */
+#define NVFP4MOE_FAST_COMBINE 0x80u
 
 const char *nvfp4moe_status_string(int status);
 int nvfp4moe_version(void);
@@ -177,6 +198,22 @@ int moe_permute_noalloc(const int32_t *topk_idx, int64_t T, int k, int E,
                         int32_t *offsets, int32_t *padded_offsets,
                         int32_t *perm, int32_t *inv_perm,
                         nvfp4moe_stream_t stream);
+
+/* Router and permutation in one pass: the top-k of the router logits is
+ * taken inside the routing-histogram kernel (each warp routes its 32 tokens
+ * and sets their expert masks directly), then the same scan and ranking as
+ * moe_permute.  The pages' token-wise path fuses its operators and keeps its
+ * metadata on the device (www.aib.vote "miniTE report", paragraph 4); the
+ * routing rule is moe_route_topk's.
+ *   logits    [T][E] FP32 router logits (finite)
+ *   topk_idx  [T][k] int32 (out), topk_w [T][k] FP32 (out)
+ *   offsets, padded_offsets, perm, inv_perm, workspace: as moe_permute
+ * Requirements: 1 <= k <= min(E, 32), E <= 1024. */
+int moe_route_permute(const float *logits, int64_t T, int E, int k,
+                      int32_t *topk_idx, float *topk_w, int32_t *offsets,
+                      int32_t *padded_offsets, int32_t *perm, int32_t *inv_perm,
+                      void *workspace, size_t workspace_bytes,
+                      nvfp4moe_stream_t stream);
 
 /* Quantize each token of x [T][K] once and write its codes, scales and
  * decode scale to all k of its rows in the padded grouped layout (the fused
@@ -287,6 +324,21 @@ int moe_expert_layer(const void *x, const int32_t *topk_idx,
                      void *workspace, size_t workspace_bytes,
                      nvfp4moe_stream_t stream);
 
+/* moe_expert_layer starting from router logits [T][E] (FP32): the top-k
+ * routing (moe_route_topk's rule) runs inside the layer's routing-histogram
+ * kernel and its result is written to topk_idx [T][k] and topk_w [T][k]
+ * (outputs, also used by the combine).  Everything else is exactly
+ * moe_expert_layer with that routing; the workspace is the same size.
+ * Requirements: those of moe_expert_layer and k <= E. */
+int moe_expert_layer_from_logits(const void *x, const float *logits,
+                                 const nvfp4moe_weights *w_gate_up,
+                                 const nvfp4moe_weights *w_down, int64_t T,
+                                 int64_t H, int64_t I, int E, int k,
+                                 int32_t *topk_idx, float *topk_w, void *y,
+                                 uint32_t flags, void *workspace,
+                                 size_t workspace_bytes,
+                                 nvfp4moe_stream_t stream);
+
 /* moe_expert_layer that also records CUDA events at its stage boundaries, so
  * a caller can time each kernel on the stream it runs on.  stage_events
  * (host array of 7 cudaEvent_t, entries may be NULL): [0] before the first
@@ -303,6 +355,56 @@ int moe_expert_layer_profiled(const void *x, const int32_t *topk_idx,
                               size_t workspace_bytes, nvfp4moe_stream_t stream,
                               void *const *stage_events);
 
+/* ------------------------------------------------------------ backward -- */
+/* Backward of the MoE expert layer in the BF16-backward mode: the pages time
+ * "NVFP4 forward, BF16 backward" at about 1.33-1.37x over BF16 (www.aib.vote
+ * "miniTE report, NVFP4 RL stability", paragraph 1) and give no formulas.
+ * This computes the exact gradient of the unquantized layer
+ *   y[t] = sum_j w[t][j] * W_dn,e (silu(g) * u),  [g | u] = W_gu,e x[t],
+ *   e = topk_idx[t][j],
+ * on its BF16 operands (the forward's quantizers act as the identity): the
+ * routing choice is not differentiated, the routing weights are.  It
+ * recomputes [g | u] from x in BF16; all products run on the tensor cores in
+ * BF16 with FP32 accumulation (tcgen05 kind::f16), intermediates (G, dG, w*h,
+ * dx rows) are stored in BF16 and dx is summed over the k slots in slot order
+ * in FP32.
+ *   x          [T][H] BF16, topk_idx [T][k] int32, topk_w [T][k] FP32
+ *   w_gate_up  [E][2I][H] BF16 (gate rows 0..I-1, up rows I..2I-1: the same
+ *              BF16 weights nvfp4_prepare_weights quantizes)
+ *   w_down     [E][H][I] BF16
+ *   dy         [T][H] BF16, the gradient of the layer output
+ *   dx         [T][H] BF16 (out)
+ *   d_topk_w   [T][k] FP32 (out): <dy[t], D[t][j]>
+ *   dw_gate_up [E][2I][H] weight gradient (out), BF16 and/or FP32 (at least
+ *              one non-NULL); dw_down [E][H][I] likewise
+ *   flags      NVFP4MOE_BWD_KEEP_DH keeps dh' = dy_rows W_dn (FP32) in the
+ *              workspace for inspection
+ *   workspace  moe_expert_layer_backward_workspace_size() bytes
+ * Requirements: H % 256 == 0, I % 256 == 0, 1 <= E <= 1024, 1 <= k <= 32. */
+#define NVFP4MOE_BWD_KEEP_DH 0x40u
+size_t moe_expert_layer_backward_workspace_size(int64_t T, int64_t H, int64_t I,
+                                                int E, int k, uint32_t flags);
+/* Byte offsets of the backward workspace's regions: [0] error word,
+ * [1] offsets, [2] padded_offsets, [3] perm, [4] inv_perm, [5] x rows and
+ * [6] dy rows (BF16, padded grouped layout, zero padding rows), [7] row
+ * weights (FP32), [8] G = x W_gu^T (BF16 [rows_cap][2I]), [9] dG (BF16),
+ * [10] w*h (BF16 [rows_cap][I]), [11] <dh', h> partials (FP32
+ * [rows_cap][I/128]), [12] dx rows (BF16, compact sorted rows), [13] dh'
+ * (FP32 [rows_cap][I], with NVFP4MOE_BWD_KEEP_DH), [14] rows_cap (a count),
+ * [15] total bytes.  `out` must hold 16 int64 (host memory). */
+int moe_expert_layer_backward_workspace_offsets(int64_t T, int64_t H, int64_t I,
+                                                int E, int k, uint32_t flags,
+                                                int64_t *out);
+int moe_expert_layer_backward(const void *x, const int32_t *topk_idx,
+                              const float *topk_w, const void *w_gate_up,
+                              const void *w_down, const void *dy, int64_t T,
+                              int64_t H, int64_t I, int E, int k, void *dx,
+                              float *d_topk_w, void *dw_gate_up_bf16,
+                              float *dw_gate_up_f32, void *dw_down_bf16,
+                              float *dw_down_f32, uint32_t flags,
+                              void *workspace, size_t workspace_bytes,
+                              nvfp4moe_stream_t stream);
+
 /* ---------------------------------------------------------- diagnostics -- */
 /* The hardware conversions the quantizer uses, exposed so their rounding can
  * be checked against the format definition: codes[i] = E2M1_rne_satfinite(y[i])
@@ -312,28 +414,18 @@ int nvfp4moe_encode_e2m1(const float *y, int64_t n, uint8_t *codes,
 int nvfp4moe_encode_ue4m3(const float *v, int64_t n, uint8_t *codes,
                           nvfp4moe_stream_t stream);
 
-/* Tensor-core throughput probe: `grid` CTAs (one per SM when grid equals the
- * SM count) each issue `iters` K-steps of 4 block-scaled FP4 MMAs
- * (tcgen05.mma kind::mxf4nvf4, M = 128, N = n in {128, 256}, K = 64) on
- * operands resident in shared memory, each K-step preceded by sf_a_copies
- * (0..4) and sf_b_copies (0..8) 512-byte scale-factor copies into TMEM, as
- * the grouped GEMM issues them.  Reads no global memory; cycles[grid]
- * (device, int64) receives each CTA's elapsed SM cycles.  The FLOP count is
- * grid * iters * 4 * 2*128*n*64.  mode: 0 = a K-step's copies then its
- * MMAs; 1 = each K-block's copies right before its MMA; 2 = the copies of
- * the next K-step (into a second TMEM buffer) before the current MMAs;
- * 3 = copies only; 4 = mode 0 with 4 + 8 copies issued from precomputed
- * descriptors; 5 = those copies only; 6 = four 2 KB 128x128b copies only;
- * 7 = four 1 KB 64x128b.warpx2 copies only; 8 = four warps write 48 scale
- * columns per K-step with tcgen05.st, no MMAs; 9 = mode 8 alongside the
- * MMAs of mode 0 without copies; 10 / 11 = modes 8 / 9 with the 48 words
- * per lane first read from the 6 KB of scale atoms in shared memory; 12 = the
- * MMAs of mode 0 while another warp fills 54 KB of shared memory per K-step
- * with bulk copies from global memory.  workspace: 16 bytes (error word),
- * 256 + 55296 bytes for mode 12 (the bulk copies' source). */
-int nvfp4moe_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies,
-                       int mode, int grid, long long *cycles, void *workspace,
-                       nvfp4moe_stream_t stream);
+/* Tensor-core throughput probe: the measured roofline denominator of the
+ * grouped GEMM (no counterpart on the pages).  `grid` CTAs (one per SM when
+ * grid equals the SM count) each issue `iters` K-steps of 4 block-scaled FP4
+ * MMAs (tcgen05.mma kind::mxf4nvf4, M = 128, N = 256, K = 64, 16-element
+ * UE4M3 scale blocks) on operands resident in shared memory, the GEMM's
+ * instruction and tile shape.  With scale_writes != 0, four warps meanwhile
+ * write each K-step's 48 scale columns into TMEM with tcgen05.st, as the
+ * GEMM's scale feeders do.  Reads no global memory.  cycles[grid] (device,
+ * int64) receives each CTA's elapsed SM cycles; the FLOP count is
+ * grid * iters * 4 * 2*128*256*64.  workspace: 16 bytes (error word). */
+int nvfp4moe_mma_peak(int iters, int scale_writes, int grid, long long *cycles,
+                      void *workspace, nvfp4moe_stream_t stream);
 
 /* Number of SMs of the current device (the persistent grids' size). */
 int nvfp4moe_num_sms(void);

@@ -75,6 +75,7 @@ int64_t layer_rows_cap(int64_t T, int k, int E) { return round_up(T * k + 127 * 
 struct LayerLayout {
   int64_t v[16];
   int64_t counts, local_rank;
+  int64_t y_acc;     // FP32 [T][H]: the non-strict combine's accumulator
 };
 
 LayerLayout layer_layout(int64_t T, int64_t H, int64_t I, int E, int k) {
@@ -98,6 +99,43 @@ LayerLayout layer_layout(int64_t T, int64_t H, int64_t I, int E, int k) {
   L.v[13] = c.take(R * H * 2);
   L.counts = c.take(permute_blocks(T) * E * 4);
   L.local_rank = c.take(R * 4);
+  L.y_acc = c.take(T * H * 4);
+  L.v[14] = cap;
+  L.v[15] = c.off;
+  return L;
+}
+
+struct BwdLayout {
+  int64_t v[16];
+  int64_t counts, local_rank, ones;
+};
+
+// Workspace of the backward: [0] header, [1] offsets, [2] padded offsets,
+// [3] perm, [4] inv_perm, [5] x rows, [6] dy rows, [7] row weights, [8] G,
+// [9] dG, [10] w*h, [11] <dh', h> partials, [12] dx rows (compact), [13] dh'
+// (FP32, only with NVFP4MOE_BWD_KEEP_DH), [14] rows_cap, [15] total bytes.
+BwdLayout bwd_layout(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
+  const int64_t R = T * k;
+  const int64_t cap = layer_rows_cap(T, k, E);
+  Carve c;
+  BwdLayout L;
+  L.v[0] = c.take(kHeaderBytes);
+  L.v[1] = c.take((E + 1) * 4);
+  L.v[2] = c.take((E + 1) * 4);
+  L.v[3] = c.take(R * 4);
+  L.v[4] = c.take(R * 4);
+  L.v[5] = c.take(cap * H * 2);
+  L.v[6] = c.take(cap * H * 2);
+  L.v[7] = c.take(cap * 4);
+  L.v[8] = c.take(cap * 2 * I * 2);
+  L.v[9] = c.take(cap * 2 * I * 2);
+  L.v[10] = c.take(cap * I * 2);
+  L.v[11] = c.take(cap * (I / 128) * 4);
+  L.v[12] = c.take(R * H * 2);
+  L.v[13] = c.take((flags & NVFP4MOE_BWD_KEEP_DH) ? cap * I * 4 : 0);
+  L.counts = c.take(permute_blocks(T) * E * 4);
+  L.local_rank = c.take(R * 4);
+  L.ones = c.take(R * 4);
   L.v[14] = cap;
   L.v[15] = c.off;
   return L;
@@ -386,11 +424,14 @@ int moe_expert_layer_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, i
   return NVFP4MOE_OK;
 }
 
+// logits == nullptr: topk_idx / topk_w are the given routing.  Otherwise the
+// top-k of the router logits [T][E] is taken inside the routing-histogram
+// kernel and written to topk_idx / topk_w (outputs).
 static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float *topk_w,
                              const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down,
                              int64_t T, int64_t H, int64_t I, int E, int k, void *y, uint32_t flags,
                              void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream,
-                             void *const *events) {
+                             void *const *events, const float *logits = nullptr) {
   if (T < 0 || H <= 0 || I <= 0 || k < 1 || k > 32 || E < 1) return NVFP4MOE_ERR_INVALID_ARG;
   if (E > 1024 || H % 256 != 0 || I % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
   int rc = check_weights(w_gate_up, E, 2 * I, H);
@@ -404,10 +445,14 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   const LayerLayout L = layer_layout(T, H, I, E, k);
   if (workspace == nullptr || (int64_t)workspace_bytes < L.v[15]) return NVFP4MOE_ERR_WORKSPACE;
   const bool tok = per_token(flags);
+  const bool fast_combine = (flags & NVFP4MOE_FAST_COMBINE) != 0;
+  if (fast_combine && (flags & NVFP4MOE_STRICT)) return NVFP4MOE_ERR_INVALID_ARG;
+  if (fast_combine && H % 8 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
   const int64_t cap = L.v[14];
   cudaStream_t s = st(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   int *err = reinterpret_cast<int *>(ws + L.v[0]);
+  float *y_acc = reinterpret_cast<float *>(ws + L.y_acc);
   float *x_amax = reinterpret_cast<float *>(ws + L.v[0] + kHdrXAmax);
   float *h_amax_tensor = reinterpret_cast<float *>(ws + L.v[0] + kHdrHAmax);
   int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.v[1]);
@@ -447,6 +492,12 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   // padding rows of h start with amax 0 (the requantizer skips them)
   pp.zero_pad_rows = tok ? h_amax_rows : nullptr;
   pp.rows_cap = cap;
+  if (logits != nullptr) {
+    if (k > E) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+    pp.logits = logits;
+    pp.topk_idx_out = const_cast<int32_t *>(topk_idx);
+    pp.topk_w_out = const_cast<float *>(topk_w);
+  }
   NVFP4MOE_TRY(launch_route_count(pp, s));
   if (!tok) NVFP4MOE_TRY(launch_amax(x, T * H, 1, x_amax, s));
   NVFP4MOE_TRY(launch_route_scan(pp, s));
@@ -505,10 +556,22 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   g.amax_h = tok ? h_amax_rows : h_amax_tensor;
   g.amax_h_rows = tok ? 1 : 0;
   g.err = err;
+  const bool fused_requant = tok && (flags & NVFP4MOE_FUSED_REQUANT);
+  if (fused_requant) {
+    // 5 (fused). per-row scales: each m-tile of h is requantized inside the
+    // GEMM launch as soon as all its columns and its row amax are final
+    g.req_q = hq;
+    g.req_sf = hsf;
+    g.req_s_dec = hsd;
+    g.discard_h = (flags & NVFP4MOE_KEEP_H) ? 0 : 1;
+  }
   NVFP4MOE_TRY(launch_grouped_gemm(g, s));
   NVFP4MOE_TRY(mark(3));
 
-  // 5. requantize h with the amax the epilogue reduced (amax reuse)
+  // 5. requantize h with the amax the epilogue reduced (amax reuse): a
+  // separate pass unless it ran inside the GEMM (a per-tensor amax spans
+  // every row, so it always needs the separate pass)
+  if (!fused_requant) {
   QuantParams rq;
   rq.x = hb;
   rq.tasks = T * k;
@@ -526,6 +589,7 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   rq.padded_offsets = padded;
   rq.E = E;
   NVFP4MOE_TRY(launch_quant(rq, s));
+  }
   NVFP4MOE_TRY(mark(4));
 
   // 6. down grouped GEMM -> D (BF16, compact sorted rows)
@@ -548,11 +612,21 @@ static int expert_layer_impl(const void *x, const int32_t *topk_idx, const float
   dn.out_bf16 = d;
   dn.out_padded = 0;
   dn.err = err;
+  if (fast_combine) {
+    // non-strict: the epilogue adds w * D_row into y_acc[t] (FP32 reductions)
+    NVFP4MOE_TRY(cudaMemsetAsync(y_acc, 0, T * H * 4, s));
+    dn.out_bf16 = nullptr;
+    dn.red_y = y_acc;
+    dn.red_perm = perm;
+    dn.red_w = topk_w;
+    dn.red_k = k;
+  }
   NVFP4MOE_TRY(launch_grouped_gemm(dn, s));
   NVFP4MOE_TRY(mark(5));
 
-  // 7. weighted combine in slot order
-  NVFP4MOE_TRY(launch_combine(d, inv_perm, topk_w, T, k, H, y, s));
+  // 7. weighted combine in slot order (strict), or y = BF16(y_acc)
+  if (fast_combine) NVFP4MOE_TRY(launch_f32_to_bf16(y_acc, T * H, y, s));
+  else NVFP4MOE_TRY(launch_combine(d, inv_perm, topk_w, T, k, H, y, s));
   NVFP4MOE_TRY(mark(6));
   return NVFP4MOE_OK;
 }
@@ -574,16 +648,216 @@ int moe_expert_layer_profiled(const void *x, const int32_t *topk_idx, const floa
                            workspace_bytes, stream, stage_events);
 }
 
-int nvfp4moe_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies, int mode, int grid,
-                       long long *cycles, void *workspace, nvfp4moe_stream_t stream) {
-  if (iters < 1 || (n != 128 && n != 256) || sf_a_copies < 0 || sf_a_copies > 4 || sf_b_copies < 0 ||
-      sf_b_copies > 8 || mode < 0 || mode > 12 || grid < 1 || cycles == nullptr || workspace == nullptr)
+size_t moe_expert_layer_backward_workspace_size(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+  return (size_t)bwd_layout(T, H, I, E, k, flags).v[15];
+}
+
+int moe_expert_layer_backward_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags,
+                                                int64_t *out) {
+  if (out == nullptr || T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(T, H, I, E, k, flags);
+  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
+  return NVFP4MOE_OK;
+}
+
+int moe_expert_layer_backward(const void *x, const int32_t *topk_idx, const float *topk_w, const void *w_gate_up,
+                              const void *w_down, const void *dy, int64_t T, int64_t H, int64_t I, int E, int k,
+                              void *dx, float *d_topk_w, void *dw_gate_up_bf16, float *dw_gate_up_f32,
+                              void *dw_down_bf16, float *dw_down_f32, uint32_t flags, void *workspace,
+                              size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (T < 0 || H <= 0 || I <= 0 || k < 1 || k > 32 || E < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || H % 256 != 0 || I % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return NVFP4MOE_OK;
+  if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || w_gate_up == nullptr || w_down == nullptr ||
+      dy == nullptr || dx == nullptr || d_topk_w == nullptr ||
+      (dw_gate_up_bf16 == nullptr && dw_gate_up_f32 == nullptr) || (dw_down_bf16 == nullptr && dw_down_f32 == nullptr))
     return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(dy) || !aligned16(dx) ||
+      !aligned16(dw_gate_up_bf16) || !aligned16(dw_gate_up_f32) || !aligned16(dw_down_bf16) ||
+      !aligned16(dw_down_f32) || !aligned16(workspace))
+    return NVFP4MOE_ERR_MISALIGNED;
+  const BwdLayout L = bwd_layout(T, H, I, E, k, flags);
+  if (workspace == nullptr || (int64_t)workspace_bytes < L.v[15]) return NVFP4MOE_ERR_WORKSPACE;
+  const int64_t cap = L.v[14];
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int *err = reinterpret_cast<int *>(ws + L.v[0]);
+  int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.v[1]);
+  int32_t *padded = reinterpret_cast<int32_t *>(ws + L.v[2]);
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.v[3]);
+  int32_t *inv_perm = reinterpret_cast<int32_t *>(ws + L.v[4]);
+  void *x_rows = ws + L.v[5];
+  void *dy_rows = ws + L.v[6];
+  float *w_rows = reinterpret_cast<float *>(ws + L.v[7]);
+  void *g = ws + L.v[8];
+  void *dg = ws + L.v[9];
+  void *hw = ws + L.v[10];
+  float *dw_part = reinterpret_cast<float *>(ws + L.v[11]);
+  void *dx_rows = ws + L.v[12];
+  float *dh_keep = (flags & NVFP4MOE_BWD_KEEP_DH) ? reinterpret_cast<float *>(ws + L.v[13]) : nullptr;
+  float *ones = reinterpret_cast<float *>(ws + L.ones);
+  NVFP4MOE_TRY(cudaMemsetAsync(ws + L.v[0], 0, kHeaderBytes, s));
+
+  // routing metadata: offsets, padded offsets, perm, inv_perm
+  PermuteParams pp;
+  pp.topk_idx = topk_idx;
+  pp.T = T;
+  pp.k = k;
+  pp.E = E;
+  pp.block_counts = reinterpret_cast<int32_t *>(ws + L.counts);
+  pp.local_rank = reinterpret_cast<int32_t *>(ws + L.local_rank);
+  pp.offsets = offsets;
+  pp.padded_offsets = padded;
+  pp.perm = perm;
+  pp.inv_perm = inv_perm;
+  pp.err = err;
+  NVFP4MOE_TRY(launch_route_count(pp, s));
+  NVFP4MOE_TRY(launch_route_scan(pp, s));
+  NVFP4MOE_TRY(launch_route_rank(pp, s));
+
+  // rows of x and dy in the padded grouped layout, row weights, ones
+  BwdGatherParams gp;
+  gp.x = x;
+  gp.dy = dy;
+  gp.topk_w = topk_w;
+  gp.topk_idx = topk_idx;
+  gp.perm = perm;
+  gp.offsets = offsets;
+  gp.padded_offsets = padded;
+  gp.T = T;
+  gp.H = H;
+  gp.rows_cap = cap;
+  gp.k = k;
+  gp.E = E;
+  gp.x_rows = x_rows;
+  gp.dy_rows = dy_rows;
+  gp.w_rows = w_rows;
+  gp.ones = ones;
+  NVFP4MOE_TRY(launch_bwd_gather(gp, s));
+
+  Bf16GemmArgs base;
+  base.offsets = offsets;
+  base.padded_offsets = padded;
+  base.E = E;
+  base.rows_cap = cap;
+  base.err = err;
+  // G = x_rows W_gu^T (the forward's gate_up product, recomputed in BF16)
+  Bf16GemmArgs g1 = base;
+  g1.mode = kBfRows;
+  g1.a = x_rows;
+  g1.b = w_gate_up;
+  g1.b_mn = 0;
+  g1.N = 2 * I;
+  g1.K = H;
+  g1.out_bf16 = g;
+  g1.out_padded = 1;
+  NVFP4MOE_TRY(launch_bf16_gemm(g1, s));
+  // dh' = dy_rows W_dn; epilogue: SwiGLU backward -> dG, w*h, <dh', h> partials
+  Bf16GemmArgs g2 = base;
+  g2.mode = kBfRows;
+  g2.a = dy_rows;
+  g2.b = w_down;
+  g2.b_mn = 1;
+  g2.N = I;
+  g2.K = H;
+  g2.epilogue = kBfSwiGLUBwd;
+  g2.g_u = g;
+  g2.w_rows = w_rows;
+  g2.d_gu = dg;
+  g2.hw = hw;
+  g2.dw_part = dw_part;
+  g2.out_f32 = dh_keep;
+  NVFP4MOE_TRY(launch_bf16_gemm(g2, s));
+  // dx rows = dG W_gu (compact sorted rows), then dx[t] = sum_j dx_rows[inv_perm[t][j]]
+  Bf16GemmArgs g3 = base;
+  g3.mode = kBfRows;
+  g3.a = dg;
+  g3.b = w_gate_up;
+  g3.b_mn = 1;
+  g3.N = H;
+  g3.K = 2 * I;
+  g3.out_bf16 = dx_rows;
+  g3.out_padded = 0;
+  NVFP4MOE_TRY(launch_bf16_gemm(g3, s));
+  NVFP4MOE_TRY(launch_combine(dx_rows, inv_perm, ones, T, k, H, dx, s));
+  // d topk_w[t][j] = <dy[t], D[t][j]> = sum of the row's partials
+  NVFP4MOE_TRY(launch_bwd_dw(dw_part, I / 128, inv_perm, topk_idx, offsets, padded, T, k, E, d_topk_w, s));
+  // dW_dn,e = sum over the group's rows of dy_r^T (w h)_r
+  Bf16GemmArgs g4 = base;
+  g4.mode = kBfWgrad;
+  g4.a = dy_rows;
+  g4.b = hw;
+  g4.M = H;
+  g4.N = I;
+  g4.out_bf16 = dw_down_bf16;
+  g4.out_f32 = dw_down_f32;
+  NVFP4MOE_TRY(launch_bf16_gemm(g4, s));
+  // dW_gu,e = sum over the group's rows of dG_r^T x_r
+  Bf16GemmArgs g5 = base;
+  g5.mode = kBfWgrad;
+  g5.a = dg;
+  g5.b = x_rows;
+  g5.M = 2 * I;
+  g5.N = H;
+  g5.out_bf16 = dw_gate_up_bf16;
+  g5.out_f32 = dw_gate_up_f32;
+  NVFP4MOE_TRY(launch_bf16_gemm(g5, s));
+  return NVFP4MOE_OK;
+}
+
+int moe_route_permute(const float *logits, int64_t T, int E, int k, int32_t *topk_idx, float *topk_w,
+                      int32_t *offsets, int32_t *padded_offsets, int32_t *perm, int32_t *inv_perm, void *workspace,
+                      size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (T < 0 || k < 1 || E < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32 || k > E) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (offsets == nullptr || padded_offsets == nullptr ||
+      (T > 0 && (logits == nullptr || topk_idx == nullptr || topk_w == nullptr || perm == nullptr ||
+                 inv_perm == nullptr)))
+    return NVFP4MOE_ERR_INVALID_ARG;
+  const PermuteLayout L = permute_layout(T, k, E);
+  if (workspace == nullptr || (int64_t)workspace_bytes < L.total) return NVFP4MOE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  NVFP4MOE_TRY(cudaMemsetAsync(ws + L.hdr, 0, 16, s));
+  PermuteParams p;
+  p.topk_idx = topk_idx;
+  p.T = T;
+  p.k = k;
+  p.E = E;
+  p.block_counts = reinterpret_cast<int32_t *>(ws + L.counts);
+  p.local_rank = reinterpret_cast<int32_t *>(ws + L.local_rank);
+  p.offsets = offsets;
+  p.padded_offsets = padded_offsets;
+  p.perm = perm;
+  p.inv_perm = inv_perm;
+  p.err = reinterpret_cast<int *>(ws + L.hdr);
+  p.logits = logits;
+  p.topk_idx_out = topk_idx;
+  p.topk_w_out = topk_w;
+  NVFP4MOE_TRY(launch_route_count(p, s));
+  NVFP4MOE_TRY(launch_route_scan(p, s));
+  NVFP4MOE_TRY(launch_route_rank(p, s));
+  return NVFP4MOE_OK;
+}
+
+int moe_expert_layer_from_logits(const void *x, const float *logits, const nvfp4moe_weights *w_gate_up,
+                                 const nvfp4moe_weights *w_down, int64_t T, int64_t H, int64_t I, int E, int k,
+                                 int32_t *topk_idx, float *topk_w, void *y, uint32_t flags, void *workspace,
+                                 size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (T > 0 && logits == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  return expert_layer_impl(x, topk_idx, topk_w, w_gate_up, w_down, T, H, I, E, k, y, flags, workspace,
+                           workspace_bytes, stream, nullptr, logits);
+}
+
+int nvfp4moe_mma_peak(int iters, int scale_writes, int grid, long long *cycles, void *workspace,
+                      nvfp4moe_stream_t stream) {
+  if (iters < 1 || grid < 1 || cycles == nullptr || workspace == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
   cudaStream_t s = st(stream);
   NVFP4MOE_TRY(cudaMemsetAsync(workspace, 0, 16, s));
-  return cuda_rc(launch_mma_probe(iters, n, sf_a_copies, sf_b_copies, mode, cycles,
-                                  static_cast<int *>(workspace),
-                                  static_cast<const uint8_t *>(workspace) + 256, grid, s));
+  return cuda_rc(launch_mma_peak(iters, scale_writes ? 1 : 0, cycles, static_cast<int *>(workspace), grid, s));
 }
 
 int nvfp4moe_num_sms(void) { return num_sms(); }

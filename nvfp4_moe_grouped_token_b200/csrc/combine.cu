@@ -100,7 +100,26 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
   }
 }
 
+// y = BF16(acc), 8 values per thread (the non-strict combine's last step).
+__global__ void k_f32_to_bf16(const float4 *__restrict__ src, int64_t n8, uint4 *__restrict__ dst) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldg(src + 2 * i), b = __ldg(src + 2 * i + 1);
+    dst[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_f32_to_bf16(const float *src, int64_t n, void *dst, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  if (n % 8 != 0) return cudaErrorInvalidValue;
+  int64_t blocks = (n / 8 + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  k_f32_to_bf16<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(src), n / 8,
+                                                  static_cast<uint4 *>(dst));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const void *d, const int32_t *inv_perm, const float *w, int64_t T, int k,
                            int64_t H, void *y, cudaStream_t s) {

@@ -7,31 +7,46 @@
 // read on the device from padded_offsets, so the host never synchronizes.
 //
 // Design (B200):
-//   * tile 128 x BN x 256 (M x N x K elements); BN = 256 with one TMEM
-//     accumulator for both GEMMs (the SwiGLU epilogue needs the gate and up
-//     halves of a 256-wide tile; BN = 128 with two accumulators measured
-//     slower for down: twice the A re-reads).  A rows come
-//     from the padded grouped layout, where every expert's group starts on a
-//     128-row boundary, so a tile never straddles two experts.
-//   * warp 4, one thread: TMA producer.  Per K-step it loads the A tile
-//     (16 KB) and the B tile (32 KB) with 128-byte-swizzled tensor copies,
-//     and the scales with plain bulk copies: A's 2 KB (the K-step-major
-//     layout [K/256][rows][16] puts a tile's 128 rows x 16 scales of one
-//     K-step in one contiguous run) and B's 4 KB (prepared in the MMA atom
-//     layout), into a shared-memory ring.
-//   * warp 1, one thread: copies the scale factors into TMEM (tcgen05.cp) and
-//     issues tcgen05.mma kind::mxf4nvf4 with 16-element UE4M3 scale blocks,
-//     FP32 accumulators in TMEM (256 columns), then commits the stage back to
-//     the producer and, after the last K-step, the accumulator to the epilogue.
-//   * warps 2-9: epilogue.  Each warp reads its 32-lane quarter of the
-//     accumulator (half of the columns), releases TMEM at once so the next
-//     tile's MMAs overlap the rest of the epilogue, scales by
-//     S_dec_a(row) * S_dec_w(expert) and stores BF16 / FP32 rows, or applies
-//     SwiGLU (gate and up columns sit in the two 128-column halves of the
-//     tile), stores h in BF16 and max-reduces |h| for the requantization.
-//   * persistent grid: one CTA per SM walks tiles t = blockIdx.x, +gridDim.x,
-//     ...; t enumerates (m-tile, n-tile) with n fastest so CTAs working at the
-//     same time share A tiles and expert weights through L2.
+//   * tile 128 x 256 x 256 (M x N x K elements) with one 256-column TMEM
+//     accumulator, for both GEMMs (the SwiGLU epilogue needs the gate and up
+//     halves of a 256-wide tile).  A rows come from the padded grouped
+//     layout, where every expert's group starts on a 128-row boundary, so a
+//     tile never straddles two experts.
+//   * 16 warps in four warpgroups:
+//       warps 0-3   scale feeders: per K-step, each reads its 32-row quarter of
+//                   the stage's scales from shared memory, rebuilds the MMA
+//                   atom order in registers and writes the stage's TMEM scale
+//                   slot with tcgen05.st;
+//       warp 4      TMA producer (one thread): A tile (16 KB) and B tile
+//                   (32 KB) by 128-byte-swizzled tensor copies, A's 2 KB of
+//                   K-step-major scales and B's 4 KB of scale atoms by bulk
+//                   copies, into a 3-stage shared-memory ring;
+//       warp 5      MMA issuer (one thread): tcgen05.mma kind::mxf4nvf4 with
+//                   16-element UE4M3 scale blocks read from TMEM, FP32
+//                   accumulation in TMEM; commits each stage back to the
+//                   producer and the finished accumulator to the epilogue;
+//       warps 6-7   requantization workers (SwiGLU GEMM with fused requant);
+//       warps 8-15  epilogue: each reads its 32-lane quarter of the
+//                   accumulator (half of the columns), releases TMEM at once
+//                   so the next tile's MMAs overlap the rest of the epilogue,
+//                   scales by S_dec_a(row) * S_dec_w(expert) and stores BF16
+//                   (or FP32) rows through TMA tensor stores, or applies
+//                   SwiGLU (gate and up sit in the two 128-column halves of a
+//                   tile), stores h in BF16 and max-reduces |h| per row.
+//   * fused requantization (per-row scales): the CTA walks its m-tiles with
+//     all their n-tiles in a row, so a row of h -- and its amax -- is
+//     complete inside one CTA once the m-tile's last n-tile is stored.  The
+//     epilogue warps then count the m-tile done (shared memory); the two
+//     worker warps (and, once their tiles are over, the epilogue warps) copy
+//     the m-tile's h back from L2 into shared memory in pieces, NVFP4-quantize
+//     it with the row amax (amax reuse) and write codes, scales and S_dec,
+//     while the MMAs run the next m-tile -- so h makes no separate trip
+//     through HBM for the requantization.  Optionally the h lines are then
+//     dropped from L2 without a write-back (discard.global.L2).
+//   * persistent grid, one CTA per SM.  Without the fused requantization the
+//     CTA walks tiles t = blockIdx.x, +gridDim.x, ... over (m-tile, n-tile)
+//     with n fastest, so CTAs working at the same time share A tiles and
+//     expert weights through L2.
 //   * every wait is bounded (common.cuh); a timeout records an error word and
 //     the CTA drains its in-flight copies and MMAs before freeing TMEM.
 #include <cudaTypedefs.h>
@@ -48,19 +63,26 @@ namespace {
 
 constexpr int BM = 128, BK = 256;
 // 16 warps in four warpgroups: 0-3 scale feeders (one per TMEM lane quarter),
-// 4 the TMA producer, 5 the MMA issuer (6-7 idle), 8-15 the epilogue.
-// setmaxnreg moves registers from the first two warpgroups to the epilogue:
-// 128 * 96 + 128 * 56 + 256 * 176 = 64512 <= 65536 launched (512 * 128).
+// 4 the TMA producer, 5 the MMA issuer, 6-7 the requantization workers, 8-15
+// the epilogue.  setmaxnreg moves registers from the first two warpgroups to
+// the epilogue: 128 * 88 + 128 * 72 + 256 * 176 = 65536 launched (512 * 128).
 constexpr int kFeedWarps = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 8;
+constexpr int kWorkWarp0 = 6;
 constexpr int kThreads = 512;
-constexpr uint32_t kRegsFeed = 96, kRegsCtl = 56, kRegsEpi = 176;
+constexpr uint32_t kRegsFeed = 88, kRegsCtl = 72, kRegsEpi = 176;
 static_assert(128 * kRegsFeed + 128 * kRegsCtl + 256 * kRegsEpi <= 65536, "register split");
 constexpr uint32_t kTmemCols = 512;
 // Epilogue staging: per epilogue warp two 2 KB buffers of 32 rows x 32 BF16
 // (64-byte swizzle), drained to global memory by TMA tensor stores.
 constexpr int kStagingPerWarp = 4096;
+// Rows per slab of h: the unit of the fused requantization.
+constexpr int kSlabRows = 32;
+// Bytes of h a worker warp copies into shared memory per step (a multiple of
+// 128, so a group of four 16-element blocks never straddles two pieces), two
+// pieces in flight per warp.
+constexpr uint32_t kReqPiece = 5632;
 
 template <int BN_, int STAGES_, int ACC_>
 struct Cfg {
@@ -81,7 +103,11 @@ struct Cfg {
   static constexpr int kChunks = kColsPerWarp / 32;
   static constexpr size_t kStagingOff = (size_t)STAGES * kStageBytes;
   static constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
-  static constexpr size_t kSmemFixed = kBarrierOff + 1024 + 256;
+  // fused requantization: each worker warp stages h through two buffers
+  static constexpr size_t kReqOff = kBarrierOff + 512;   // barriers and flags: 512 bytes
+  static constexpr size_t kOffsetsOff = kReqOff + 4 * (size_t)kReqPiece;
+  // + up to 1023 bytes lost to aligning the dynamic shared memory to 1 KB
+  static constexpr size_t kSmemFixed = kOffsetsOff + 1024;
   static constexpr size_t kSmemMax = kSmemFixed + (size_t)8 * 1025;   // + offsets of E <= 1024
   // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
   // UE4M3 scales (bit 23 = 0), N >> 3 at bit 17, M >> 4 at bit 24, dense, K = 64.
@@ -126,6 +152,213 @@ __device__ __forceinline__ float fmax_abs_bf16(float m, uint32_t packed) {
   return fmaxf(m, fmaxf(fabsf(bf16_lo(packed)), fabsf(bf16_hi(packed))));
 }
 
+__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t *p) {
+  return *reinterpret_cast<const volatile uint32_t *>(p);
+}
+
+// Bounded spin on a shared-memory word until it equals `want`.
+__device__ __forceinline__ bool wait_u32_eq(const uint32_t *p, uint32_t want, volatile int *abort_flag,
+                                            int *err, int where) {
+  if (ld_volatile_u32(p) == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (ld_volatile_u32(p) == want) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        set_device_error(err, kDevTimeout, where);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Fused requantization bookkeeping, per CTA, in shared memory:
+//   mt_done     +1 by each epilogue warp once its h stores and row-amax
+//               updates for one of the CTA's m-tiles are complete (so the j-th
+//               m-tile is ready when mt_done >= 8 (j + 1))
+//   slab_next   slabs of the CTA's m-tiles claimed so far (4 per m-tile)
+// Claim the CTA's next slab (one thread): returns its index k (m-tile k / 4
+// of this CTA, slab k % 4 of it) once that m-tile is ready, or -1 when none
+// is left (or the kernel is aborting).
+__device__ __forceinline__ int64_t claim_slab(uint32_t *slab_next, const uint32_t *mt_done, int64_t nslabs,
+                                              volatile int *abort_flag, int *err) {
+  const int64_t k = atomicAdd(slab_next, 1u);
+  if (k >= nslabs) return -1;
+  const uint32_t need = (uint32_t)(kEpiWarps * (k / (BM / kSlabRows) + 1));
+  if (ld_volatile_u32(mt_done) >= need) return k;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(200);
+    if (ld_volatile_u32(mt_done) >= need) return k;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return -1;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        set_device_error(err, kDevTimeout, 402);
+        *abort_flag = 1;
+        return -1;
+      }
+    }
+  }
+}
+
+// NVFP4 quantization of one 16-element block of BF16 values (two uint4) under
+// the row's S_enc, one binary32 operation per step, round to nearest even:
+// sf = UE4M3((bamax / 6) * S_enc), code = E2M1(x * (S_enc / sf)), all +0
+// when sf == 0.
+__device__ __forceinline__ uint32_t encode_block16(const uint4 &v0, const uint4 &v1, float s_enc,
+                                                   uint2 &codes) {
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
+#pragma unroll
+  for (int j = 1; j < 8; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
+  const float bamax = fmaxf(__low2float(m2), __high2float(m2));
+  const uint32_t sfc = cvt_ue4m3(__fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc));
+  codes = make_uint2(0, 0);
+  if (sfc != 0) {
+    const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      y[2 * j] = __fmul_rn(bf16_lo(w[j]), rr);
+      y[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), rr);
+    }
+    codes.x = cvt_e2m1x8(y);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      y[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), rr);
+      y[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), rr);
+    }
+    codes.y = cvt_e2m1x8(y);
+  }
+  return sfc;
+}
+
+// Shared-memory staging of one warp for the requantization: two buffers of
+// `piece` bytes with one mbarrier each; `loads[i]` counts the copies that
+// buffer i has received (its barrier's phase), across slabs.
+struct ReqStage {
+  uint8_t *buf[2];
+  uint64_t *bar[2];
+  uint32_t piece;
+  uint32_t loads[2];
+};
+
+// Requantize the 32 rows of h slab `slab` (rows slab*32 ..) with their
+// per-row amax (reduced by the epilogue: amax reuse), one warp.  The slab's
+// 32 rows are one contiguous run of 32 * I BF16; it is copied into shared
+// memory in pieces (bulk copies, the next piece landing while this one is
+// encoded), so the warp keeps whole pieces in flight instead of one row.  A
+// row whose amax is 0 (a padding row, or an all-zero row) gets zero codes,
+// zero scales and S_dec = 1.  Writes codes [rows][I/2], scales in the
+// K-step-major layout and the row S_dec; then, if asked, drops the slab's h
+// lines from L2 without writing them back.
+__device__ __noinline__ void requant_slab(const GemmArgs &a, int32_t slab, int lane, ReqStage &rs,
+                                          volatile int *abort_flag) {
+  const int64_t I = a.N >> 1;
+  const uint32_t nblk = (uint32_t)(I >> 4);
+  const int64_t row0 = (int64_t)slab * kSlabRows;
+  const uint8_t *src = reinterpret_cast<const uint8_t *>(static_cast<const __nv_bfloat16 *>(a.out_bf16) + row0 * I);
+  const uint32_t total = (uint32_t)(kSlabRows * I * 2);
+  const uint32_t npieces = (total + rs.piece - 1) / rs.piece;
+  // lane r: the global scales of row row0 + r
+  float my_enc, my_dec;
+  const float my_amax = __ldcg(a.amax_h + row0 + lane);
+  global_scales(my_amax, my_enc, my_dec);
+  a.req_s_dec[row0 + lane] = my_dec;
+  // the h just published by other CTAs is read through the async proxy
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  auto issue = [&](uint32_t pc) {
+    if (lane == 0) {
+      const uint32_t bi = pc & 1u;
+      const uint32_t off = pc * rs.piece;
+      const uint32_t n = total - off < rs.piece ? total - off : rs.piece;
+      mbar_arrive_expect_tx(rs.bar[bi], n);
+      bulk_load(rs.buf[bi], src + off, n, rs.bar[bi]);
+    }
+  };
+  issue(0);
+  for (uint32_t pc = 0; pc < npieces; ++pc) {
+    const uint32_t bi = pc & 1u;
+    if (pc + 1 < npieces) issue(pc + 1);     // into the buffer read in the previous step
+    const bool ok = mbar_wait_bounded(rs.bar[bi], rs.loads[bi] & 1u, abort_flag, a.err, 403);
+    ++rs.loads[bi];
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (pc + 1 < npieces) {               // let the copy in flight land before leaving
+        int never = 0;
+        mbar_wait_bounded(rs.bar[bi ^ 1u], rs.loads[bi ^ 1u] & 1u, &never, a.err, 404);
+        ++rs.loads[bi ^ 1u];
+      }
+      return;
+    }
+    const uint32_t off = pc * rs.piece;
+    const uint32_t n = total - off < rs.piece ? total - off : rs.piece;
+    const uint32_t nb = n / 32;            // 16-element blocks in this piece
+    const uint4 *pbuf = reinterpret_cast<const uint4 *>(rs.buf[bi]);
+    // two blocks per lane per step (blk and blk + 32): independent chains
+    // the scheduler can interleave
+    for (uint32_t j0 = 0; j0 < nb; j0 += 64) {
+      uint2 codes[2];
+      uint32_t sfc[2], rr[2], bb[2];
+      bool valid[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t blk = j0 + 32 * u + (uint32_t)lane;
+        valid[u] = blk < nb;
+        const uint32_t gb = off / 32 + blk;    // block index inside the slab
+        rr[u] = valid[u] ? gb / nblk : 0;
+        bb[u] = gb - rr[u] * nblk;
+      }
+      float s_enc[2];
+      bool live[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        s_enc[u] = __shfl_sync(0xffffffffu, my_enc, (int)rr[u]);
+        live[u] = __shfl_sync(0xffffffffu, my_amax, (int)rr[u]) > 0.0f;
+      }
+      uint4 v[2][2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        v[u][0] = make_uint4(0, 0, 0, 0);
+        v[u][1] = v[u][0];
+        if (valid[u] && live[u]) {
+          const uint32_t blk = j0 + 32 * u + (uint32_t)lane;
+          v[u][0] = pbuf[blk * 2];
+          v[u][1] = pbuf[blk * 2 + 1];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) sfc[u] = encode_block16(v[u][0], v[u][1], s_enc[u], codes[u]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (j0 + 32 * u >= nb) break;          // warp-uniform
+        // the four scales of blocks 4i..4i+3 (one row: pieces and nblk are
+        // multiples of 4 blocks) sit in lanes 4i..4i+3
+        const int q4 = lane & ~3;
+        const uint32_t s0 = __shfl_sync(0xffffffffu, sfc[u], q4);
+        const uint32_t s1 = __shfl_sync(0xffffffffu, sfc[u], q4 + 1);
+        const uint32_t s2 = __shfl_sync(0xffffffffu, sfc[u], q4 + 2);
+        const uint32_t s3 = __shfl_sync(0xffffffffu, sfc[u], q4 + 3);
+        if (valid[u]) {
+          const int64_t row = row0 + rr[u];
+          const uint32_t b = bb[u];
+          *reinterpret_cast<uint2 *>(a.req_q + row * (I >> 1) + (int64_t)b * 8) = codes[u];
+          if ((lane & 3) == 0)
+            *reinterpret_cast<uint32_t *>(a.req_sf + (((int64_t)(b >> 4) * a.rows_cap + row) * 16 + (b & 15))) =
+                s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+      }
+    }
+    __syncwarp();                            // this buffer is free for piece pc + 2
+  }
+  if (a.discard_h) {
+    const int64_t lines = (int64_t)total / 128;
+    for (int64_t i = lane; i < lines; i += 32)
+      asm volatile("discard.global.L2 [%0], 128;" ::"l"(src + i * 128) : "memory");
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_constant__ KParams P) {
   constexpr int BN = C::BN, STAGES = C::STAGES, ACC = C::ACC;
@@ -141,11 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *never = reinterpret_cast<int *>(tmem_slot + 2);   // an abort flag nothing raises
-  int32_t *s_pad = reinterpret_cast<int32_t *>(smem + C::kBarrierOff + 256);
+  uint64_t *req_bar = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 128);   // [2 workers][2]
+  uint32_t *mt_done = reinterpret_cast<uint32_t *>(smem + C::kBarrierOff + 320);
+  uint32_t *slab_next = mt_done + 1;
+  int32_t *s_pad = reinterpret_cast<int32_t *>(smem + C::kOffsetsOff);
   int32_t *s_off = s_pad + (P.a.E + 1);
 
   const GemmArgs &a = P.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // requantize h inside this launch (SwiGLU epilogue, per-row amax)
+  const bool fused_requant = a.epilogue == kEpiSwiGLU && a.req_q != nullptr && a.amax_h != nullptr &&
+                             a.amax_h_rows != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -158,6 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       mbar_init(&acc_empty[s], kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&req_bar[i], 1);
+    *mt_done = 0;
+    *slab_next = 0;
     *abort_flag = 0;
     *never = 0;
     fence_mbarrier_init();
@@ -191,8 +433,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   const int64_t k_atoms = a.K >> 6;      // 512-byte scale atoms per 128 rows
 
   const uint32_t smem0 = smem_u32(smem);
-  // K-steps of this CTA: its tiles blockIdx.x, +gridDim.x, ... times kt_count
-  const int64_t my_tiles = total > (int64_t)blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  // Tile order.  Default: t = blockIdx.x, +gridDim.x, ... over (m-tile,
+  // n-tile) with n fastest, so the CTAs running together share A tiles and
+  // expert weights through L2.  With the fused requantization: m-tile-major
+  // per CTA (m-tiles blockIdx.x, +gridDim.x, ..., each with all its n-tiles in
+  // order), so every row of h is completed by one CTA.
+  const int64_t m_total = rows_used / BM;
+  const bool m_major = fused_requant;
+  const int64_t my_mtiles = m_total > (int64_t)blockIdx.x ? (m_total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t my_tiles = m_major ? my_mtiles * n_tiles
+                                   : (total > (int64_t)blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0);
+  auto tile_mn = [&](int64_t i, int64_t &mt, int &nt) {
+    if (m_major) {
+      const int64_t j = i / n_tiles;
+      mt = (int64_t)blockIdx.x + j * gridDim.x;
+      nt = (int)(i - j * n_tiles);
+    } else {
+      const int64_t t = (int64_t)blockIdx.x + i * gridDim.x;
+      mt = t / n_tiles;
+      nt = (int)(t - mt * n_tiles);
+    }
+  };
   const uint32_t steps = (uint32_t)(my_tiles * kt_count);
 
   if (warp < kFeedWarps) {
@@ -248,9 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       // step costs this thread hundreds of cycles of latency)
       uint32_t p = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const int64_t mt = t / n_tiles;
-        const int nt = (int)(t - mt * n_tiles);
+      for (int64_t i = 0; i < my_tiles && ok; ++i) {
+        int64_t mt;
+        int nt;
+        tile_mn(i, mt, nt);
         const int e = find_group(s_pad, a.E, mt * BM);
         const int32_t arow = (int32_t)(mt * BM);
         const int32_t wrow0 = (int32_t)((int64_t)e * a.N + (int64_t)nt * BN);
@@ -284,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       const uint64_t op_desc0 = smem_desc(0, 16, 1024, 2);   // K-major, 128-byte swizzle
       uint32_t st = 0, ph = 0, it = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+      for (int64_t i = 0; i < my_tiles && ok; ++i, ++it) {
         const uint32_t as = it % ACC;
         const uint32_t acc = tmem + as * BN;
         if (!mbar_wait_bounded(&acc_empty[as], ((it / ACC) & 1u) ^ 1u, abort_flag, a.err, 200)) break;
@@ -307,6 +569,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       // drain: all MMAs this thread issued have completed
       tc_commit(drain);
       mbar_wait_bounded(drain, 0, never, a.err, 202);
+    } else if (warp >= kWorkWarp0 && fused_requant) {
+      // ------------------------------------------- requantization workers
+      const int64_t nslabs = my_mtiles * (BM / kSlabRows);
+      const int wk = warp - kWorkWarp0;
+      ReqStage rs;
+      rs.buf[0] = smem + C::kReqOff + (2 * wk) * (size_t)kReqPiece;
+      rs.buf[1] = rs.buf[0] + kReqPiece;
+      rs.bar[0] = &req_bar[2 * wk];
+      rs.bar[1] = &req_bar[2 * wk + 1];
+      rs.piece = kReqPiece;
+      rs.loads[0] = rs.loads[1] = 0;
+      for (;;) {
+        int64_t k = -1;
+        if (lane == 0) k = claim_slab(slab_next, mt_done, nslabs, abort_flag, a.err);
+        k = __shfl_sync(0xffffffffu, k, 0);
+        if (k < 0) break;
+        __threadfence_block();   // pairs with the epilogue warps' release of mt_done
+        const int64_t mt = (int64_t)blockIdx.x + (k / (BM / kSlabRows)) * gridDim.x;
+        requant_slab(a, (int32_t)(mt * (BM / kSlabRows) + k % (BM / kSlabRows)), lane, rs, abort_flag);
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
@@ -334,9 +616,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       }
       ++chunk_id;
     };
-    for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const int64_t mt = t / n_tiles;
-      const int nt = (int)(t - mt * n_tiles);
+    // fused requantization: the warp's |h| maxima of a row are kept across
+    // the n-tiles of an m-tile and folded into the row amax at its last
+    // n-tile.  One tile later (its older bulk groups are then complete) lane
+    // 0 makes the m-tile's h stores and amax updates visible and bumps
+    // mt_done; the warp barrier before it orders every lane's updates.
+    auto signal_mtile = [&](bool keep_two) {
+      if (lane == 0) {
+        if (keep_two) bulk_wait_group<2>(); else bulk_wait_group<0>();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence_block();
+        atomicAdd(mt_done, 1u);
+      }
+      __syncwarp();
+    };
+    float row_amax = 0.0f;
+    bool pending_mtile = false;
+    for (int64_t i = 0; i < my_tiles; ++i, ++it) {
+      int64_t mt;
+      int nt;
+      tile_mn(i, mt, nt);
       const int64_t row0 = mt * BM;
       const int e = find_group(s_pad, a.E, row0);
       const int64_t g_pad = s_pad[e];
@@ -399,7 +698,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
           store_box(hp[c], (int32_t)(nt * 128 + half * 64 + c * 32), (int32_t)(row0 + quad * 32));
         if (a.amax_h != nullptr) {
           if (a.amax_h_rows) {
-            if (valid) atomicMax(reinterpret_cast<unsigned int *>(a.amax_h + prow), __float_as_uint(m));
+            if (!fused_requant) {
+              if (valid) atomicMax(reinterpret_cast<unsigned int *>(a.amax_h + prow), __float_as_uint(m));
+            } else {
+              row_amax = fmaxf(row_amax, m);
+              __syncwarp();
+              // this tile's two boxes are the newest bulk groups
+              if (pending_mtile) signal_mtile(true);
+              pending_mtile = false;
+              if (nt == n_tiles - 1) {
+                if (valid) atomicMax(reinterpret_cast<unsigned int *>(a.amax_h + prow), __float_as_uint(row_amax));
+                row_amax = 0.0f;
+                pending_mtile = true;
+              }
+            }
           } else {
             float mm = valid ? m : 0.0f;
 #pragma unroll
@@ -407,6 +719,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
             if (lane == 0 && mm > 0.0f)
               atomicMax(reinterpret_cast<unsigned int *>(a.amax_h), __float_as_uint(mm));
           }
+        }
+      } else if (a.red_y != nullptr) {
+        // non-strict combine: y[t] += w[t][j] * D_row in FP32 reductions, in
+        // whatever order the tiles finish (not bitwise reproducible)
+        if (valid) {
+          const int32_t slot = __ldg(a.red_perm + g_off + rel);
+          const float wgt = __fmul_rn(__ldg(a.red_w + slot), scale);
+          float *dst = a.red_y + (int64_t)(slot / a.red_k) * a.N + (int64_t)nt * BN + half * C::kColsPerWarp;
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c * 32 + i),
+                           "f"(__fmul_rn(__uint_as_float(v[c][i]), wgt)), "f"(__fmul_rn(__uint_as_float(v[c][i + 1]), wgt)),
+                           "f"(__fmul_rn(__uint_as_float(v[c][i + 2]), wgt)), "f"(__fmul_rn(__uint_as_float(v[c][i + 3]), wgt))
+                           : "memory");
         }
       } else {
         const int64_t orow = a.out_padded ? prow : g_off + rel;
@@ -444,6 +772,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
             }
           }
         }
+      }
+    }
+    if (fused_requant) {
+      if (pending_mtile) {
+        __syncwarp();
+        signal_mtile(false);
+      }
+      // then requantize this CTA's remaining slabs with the workers, staging
+      // through this warp's two (now idle) output staging buffers
+      const int64_t nslabs = my_mtiles * (BM / kSlabRows);
+      if (lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
+      ReqStage rs;
+      rs.buf[0] = stg;
+      rs.buf[1] = stg + kStagingPerWarp / 2;
+      rs.bar[0] = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 160) + 2 * ew;
+      rs.bar[1] = rs.bar[0] + 1;
+      rs.piece = kStagingPerWarp / 2;
+      rs.loads[0] = rs.loads[1] = 0;
+      if (lane == 0) {
+        mbar_init(rs.bar[0], 1);
+        mbar_init(rs.bar[1], 1);
+        fence_mbarrier_init();
+      }
+      __syncwarp();
+      for (;;) {
+        int64_t k = -1;
+        if (lane == 0) k = claim_slab(slab_next, mt_done, nslabs, abort_flag, a.err);
+        k = __shfl_sync(0xffffffffu, k, 0);
+        if (k < 0) break;
+        __threadfence_block();
+        const int64_t mt = (int64_t)blockIdx.x + (k / (BM / kSlabRows)) * gridDim.x;
+        requant_slab(a, (int32_t)(mt * (BM / kSlabRows) + k % (BM / kSlabRows)), lane, rs, abort_flag);
       }
     }
     // every tensor store this warp issued has finished before the CTA exits
@@ -485,6 +846,16 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t esize, cons
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+bool encode_2d_map(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t esize, const void *base,
+                   uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows,
+                   CUtensorMapSwizzle swizzle) {
+  return encode_2d(map, dtype, esize, base, inner, rows, box_inner, box_rows, swizzle);
+}
+
+namespace {
 
 template <class C>
 cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
@@ -528,8 +899,8 @@ cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
 
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
   if (a.rows_cap <= 0) return cudaSuccess;
-  // the SwiGLU epilogue reads gate and up from the two halves of a 256-wide
-  // tile; plain stores use 128-wide tiles with a double-buffered accumulator
+  // both GEMMs use 128 x 256 tiles with one accumulator (the SwiGLU epilogue
+  // reads gate and up from the two 128-column halves of a tile)
   if (a.epilogue == kEpiSwiGLU) return launch_cfg<CfgGateUp>(a, s);
   return launch_cfg<CfgDown>(a, s);
 }

@@ -1,0 +1,499 @@
+// Persistent BF16 grouped GEMM over the experts on tcgen05 (sm_100a): the
+// matrix products of the layer's BF16 backward.
+//
+// The pages time a mode that runs the forward in NVFP4 and the backward in
+// BF16 (www.aib.vote "miniTE report, NVFP4 RL stability", paragraph 1:
+// about 1.33-1.37x over BF16).  Its products, per expert e with G = [g | u]
+// the gate_up output, h = silu(g) u, and rows r of the expert's group:
+//   G      = x_rows W_gu,e^T          (recomputed, BF16 operands)
+//   dh'    = dy_rows W_dn,e           (dgrad of down; B is MN-major)
+//   dx_r   = dG W_gu,e                (dgrad of gate_up; B is MN-major)
+//   dW_dn,e = dy_rows^T (w h)         (wgrad: K runs over the group's rows,
+//   dW_gu,e = dG^T x_rows              both operands MN-major)
+//
+// Design (B200):
+//   * tcgen05.mma.cta_group::1.kind::f16, M = 128, N = 256, K = 16, BF16
+//     operands from shared memory, FP32 accumulation in TMEM.  With no scale
+//     factors to stage, two 256-column accumulators fill TMEM, so the
+//     epilogue of tile i overlaps the MMAs of tile i+1.
+//   * operands are loaded by 128-byte-swizzled TMA tensor copies in either
+//     orientation: K-major (a box of 64 K-elements x rows) or MN-major (boxes
+//     of 64 M/N-elements x 64 K-rows, stacked 8 KB apart along M/N); the
+//     shared-memory matrix descriptors and the instruction descriptor's
+//     transpose bits say which.  So the backward reads every tensor where it
+//     lies, with no transposed copies.
+//   * K-step of 64 elements, a 4-stage ring (A 16 KB + B 32 KB per stage).
+//   * warp 0: TMA producer (one thread); warp 1: TMEM owner and MMA issuer
+//     (one thread); warps 4-11: epilogue, two per TMEM lane quarter, each
+//     reading half of the 256 columns.
+//   * kBfRows: tiles over (m-tile, n-tile) of the padded grouped rows with n
+//     fastest; the expert of an m-tile comes from padded_offsets.
+//     kBfWgrad: tiles over (expert, m-tile, n-tile); the K loop covers the
+//     expert's rows in steps of 64 (padding rows inside a group are zero, so
+//     the step past the last row adds nothing); an empty expert's tile is
+//     written as zeros.
+//   * every wait is bounded (common.cuh).
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4moe {
+
+// Shared tensor-map helpers of the FP4 GEMM (gemm.cu).
+bool encode_2d_map(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t esize, const void *base,
+                   uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows,
+                   CUtensorMapSwizzle swizzle);
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int STAGES = 4;
+constexpr int ACC = 2;
+constexpr int kThreads = 384;
+constexpr int kEpiWarp0 = 4, kEpiWarps = 8;
+constexpr int kABytes = BM * BK * 2;          // 16 KB
+constexpr int kBBytes = BN * BK * 2;          // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kMnBox = 64 * BK * 2;           // one MN-major box: 64 elements x 64 K-rows = 8 KB
+constexpr int kStagingPerWarp = 4096;         // two 32 x 32 BF16 boxes
+constexpr size_t kStagingOff = (size_t)STAGES * kStageBytes;
+constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
+constexpr size_t kSmemBytes = kBarrierOff + 256 + 1024;   // + slack for 1 KB alignment
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// Instruction descriptor, kind::f16: FP32 accumulator (bits 4-5 = 1), A and
+// B BF16 (bits 7-9, 10-12 = 1), transpose bits 15 (A MN-major) and 16 (B
+// MN-major), N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+struct __align__(64) BParams {
+  CUtensorMap tmap_a;
+  CUtensorMap tmap_b;
+  CUtensorMap tmap_out;   // BF16 output, 32 x 32 boxes, 64-byte swizzle
+  Bf16GemmArgs a;
+};
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void stage_row(uint32_t box_addr, int lane, const uint32_t (&w)[16]) {
+  const uint32_t base = box_addr + (uint32_t)lane * 64;
+  const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    st_shared_v4(base + (((uint32_t)q ^ sw) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
+__device__ __forceinline__ int find_group_g(const int32_t *padded, int E, int64_t row) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)__ldg(padded + mid) <= row) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Tile t of the launch: expert, first row / output row block, n block, and
+// the number of 64-element K-steps.
+struct Tile {
+  int e;
+  int64_t m0;       // kBfRows: first padded row; kBfWgrad: first M index
+  int64_t n0;
+  int64_t k_rows0;  // kBfWgrad: first padded row of the group (the K origin)
+  int ksteps;
+};
+
+__device__ __forceinline__ Tile tile_of(const Bf16GemmArgs &a, int64_t t, int n_tiles, int m_tiles) {
+  Tile r;
+  if (a.mode == kBfRows) {
+    const int64_t mt = t / n_tiles;
+    r.n0 = (t - mt * n_tiles) * BN;
+    r.m0 = mt * BM;
+    r.e = find_group_g(a.padded_offsets, a.E, r.m0);
+    r.k_rows0 = 0;
+    r.ksteps = (int)(a.K / BK);
+  } else {
+    const int64_t per_e = (int64_t)m_tiles * n_tiles;
+    r.e = (int)(t / per_e);
+    const int64_t rem = t - (int64_t)r.e * per_e;
+    const int64_t mt = rem / n_tiles;
+    r.m0 = mt * BM;
+    r.n0 = (rem - mt * n_tiles) * BN;
+    r.k_rows0 = __ldg(a.padded_offsets + r.e);
+    const int64_t cnt = (int64_t)__ldg(a.offsets + r.e + 1) - __ldg(a.offsets + r.e);
+    r.ksteps = (int)((cnt + BK - 1) / BK);
+  }
+  return r;
+}
+
+__device__ __forceinline__ float silu_f(float g, float &s) {
+  s = 1.0f / (1.0f + expf(-g));
+  return g * s;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant__ BParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarrierOff);
+  uint64_t *empty = full + STAGES;
+  uint64_t *acc_full = empty + STAGES;
+  uint64_t *acc_empty = acc_full + ACC;
+  uint64_t *drain = acc_empty + ACC;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *never = reinterpret_cast<int *>(tmem_slot + 2);
+
+  const Bf16GemmArgs &a = P.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int a_mn = a.mode == kBfWgrad ? 1 : 0;
+  const int b_mn = a.mode == kBfWgrad ? 1 : a.b_mn;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < ACC; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensor_map(&P.tmap_a);
+    prefetch_tensor_map(&P.tmap_b);
+    prefetch_tensor_map(&P.tmap_out);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_tiles = (int)(a.N / BN);
+  const int m_tiles = a.mode == kBfWgrad ? (int)(a.M / BM) : 0;
+  int64_t total;
+  if (a.mode == kBfRows) {
+    int64_t rows_used = __ldg(a.padded_offsets + a.E);
+    if (rows_used > a.rows_cap) rows_used = a.rows_cap;
+    if (rows_used < 0) rows_used = 0;
+    total = (rows_used / BM) * n_tiles;
+  } else {
+    total = (int64_t)a.E * m_tiles * n_tiles;
+  }
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      uint32_t p = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = tile_of(a, t, n_tiles, m_tiles);
+        uint32_t st = p % STAGES, ph = (p / STAGES) & 1u;
+        for (int kt = 0; kt < tl.ksteps; ++kt, ++p) {
+          if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, a.err, 500)) { ok = false; break; }
+          uint8_t *sa = smem + (size_t)st * kStageBytes;
+          uint8_t *sb = sa + kABytes;
+          mbar_arrive_expect_tx(&full[st], kStageBytes);
+          if (a.mode == kBfRows) {
+            tma_load_2d(sa, &P.tmap_a, kt * BK, (int32_t)tl.m0, &full[st]);
+            if (b_mn) {
+              // B_e[n][k] = W[e][k][n]: boxes of 64 n x 64 k-rows
+              const int32_t krow = (int32_t)((int64_t)tl.e * a.K + (int64_t)kt * BK);
+#pragma unroll
+              for (int c = 0; c < BN / 64; ++c)
+                tma_load_2d(sb + c * kMnBox, &P.tmap_b, (int32_t)(tl.n0 + 64 * c), krow, &full[st]);
+            } else {
+              tma_load_2d(sb, &P.tmap_b, kt * BK, (int32_t)((int64_t)tl.e * a.N + tl.n0), &full[st]);
+            }
+          } else {
+            const int32_t krow = (int32_t)(tl.k_rows0 + (int64_t)kt * BK);
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sa + c * kMnBox, &P.tmap_a, (int32_t)(tl.m0 + 64 * c), krow, &full[st]);
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sb + c * kMnBox, &P.tmap_b, (int32_t)(tl.n0 + 64 * c), krow, &full[st]);
+          }
+          if (++st == STAGES) { st = 0; ph ^= 1u; }
+        }
+      }
+      for (uint32_t q = p > STAGES ? p - STAGES : 0; q < p; ++q)
+        mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1u, never, a.err, 501);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      // K-major: the 16-element K slice kk starts 32 bytes further in each
+      // 128-byte row (LBO unused, SBO = 1024 between 8-row groups).
+      // MN-major: slice kk starts 16 K-rows (2 KB) further; LBO = 8 KB
+      // between 64-element M/N chunks, SBO = 1024 between 8-row K groups.
+      const uint64_t dk = smem_desc(0, 16, 1024, 2);
+      const uint64_t dmn = smem_desc(0, kMnBox, 1024, 2);
+      const uint64_t da = a_mn ? dmn : dk, db = b_mn ? dmn : dk;
+      const uint32_t step_a = a_mn ? 2048u >> 4 : 32u >> 4, step_b = b_mn ? 2048u >> 4 : 32u >> 4;
+      const uint32_t idesc = idesc_bf16(a_mn, b_mn);
+      const uint32_t smem0 = smem_u32(smem);
+      uint32_t st = 0, ph = 0, it = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const Tile tl = tile_of(a, t, n_tiles, m_tiles);
+        const uint32_t as = it % ACC;
+        const uint32_t acc = tmem + as * BN;
+        if (!mbar_wait_bounded(&acc_empty[as], ((it / ACC) & 1u) ^ 1u, abort_flag, a.err, 510)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < tl.ksteps; ++kt) {
+          if (!mbar_wait_bounded(&full[st], ph, abort_flag, a.err, 511)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t a16 = (smem0 + st * (uint32_t)kStageBytes) >> 4;
+          const uint64_t b16 = a16 + kABytes / 16;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(acc, da | (a16 + kk * step_a), db | (b16 + kk * step_b), idesc, (kt | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty[st]);
+          if (++st == STAGES) { st = 0; ph ^= 1u; }
+        }
+        if (ok) tc_commit(&acc_full[as]);
+      }
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0, never, a.err, 512);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // -------------------------------------------------------- epilogue
+    const int ew = warp - kEpiWarp0;
+    const int quad = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
+    uint8_t *stg = smem + kStagingOff + (size_t)ew * kStagingPerWarp;
+    const uint32_t stg_addr = smem_u32(stg);
+    uint32_t chunk_id = 0, it = 0;
+    auto store_box = [&](const uint32_t (&w16)[16], int32_t x, int32_t y) {
+      const uint32_t box = stg_addr + (chunk_id & 1u) * 2048;
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      stage_row(box, lane, w16);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&P.tmap_out, stg + (chunk_id & 1u) * 2048, x, y);
+        bulk_commit_group();
+      }
+      ++chunk_id;
+    };
+    const int64_t rows_total = a.mode == kBfRows ? (int64_t)__ldg(a.offsets + a.E) : 0;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const Tile tl = tile_of(a, t, n_tiles, m_tiles);
+      const uint32_t as = it % ACC;
+      // rows of this lane
+      int64_t orow;            // output row index
+      bool valid = true;
+      int64_t prow = 0;        // padded row (kBfRows)
+      bool slab_full = true;
+      int64_t slab_row = 0;
+      if (a.mode == kBfRows) {
+        const int64_t g_pad = __ldg(a.padded_offsets + tl.e);
+        const int64_t g_off = __ldg(a.offsets + tl.e);
+        const int64_t g_cnt = (int64_t)__ldg(a.offsets + tl.e + 1) - g_off;
+        const int64_t rel = tl.m0 - g_pad + quad * 32 + lane;
+        valid = rel < g_cnt && g_off + rel < rows_total;
+        prow = tl.m0 + quad * 32 + lane;
+        orow = a.out_padded ? prow : g_off + rel;
+        slab_full = a.out_padded || (tl.m0 - g_pad) + quad * 32 + 32 <= g_cnt;
+        slab_row = a.out_padded ? tl.m0 + quad * 32 : g_off + (tl.m0 - g_pad) + quad * 32;
+      } else {
+        orow = (int64_t)tl.e * a.M + tl.m0 + quad * 32 + lane;
+        slab_row = (int64_t)tl.e * a.M + tl.m0 + quad * 32;
+      }
+      float wr = 0.0f;
+      if (a.epilogue == kBfSwiGLUBwd) wr = __ldg(a.w_rows + prow);
+
+      if (!mbar_wait_bounded(&acc_full[as], (it / ACC) & 1u, abort_flag, a.err, 520)) break;
+      tc_fence_after();
+      // Chunk by chunk (32 columns): with two accumulators the MMAs of the
+      // next tile run in the other one, so this one is released after the
+      // last chunk is read.  An empty expert's tile (no K-steps) is zeros.
+      const bool zero_tile = tl.ksteps == 0;
+      const int64_t col0 = tl.n0 + half * 128;
+      const int64_t I = a.N;
+      float dwp = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        if (!zero_tile) {
+          tmem_ld_32cols(tlane + as * BN + half * 128 + c * 32, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (c == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[as]);
+        }
+        if (a.epilogue == kBfStore) {
+          if (a.out_bf16 != nullptr) {
+            uint32_t w16[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w16[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            if (slab_full) {
+              store_box(w16, (int32_t)(col0 + c * 32), (int32_t)slab_row);
+            } else if (valid) {
+              uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_bf16) + orow * a.N +
+                                                     col0 + c * 32);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+            }
+          }
+          if (a.out_f32 != nullptr && valid) {
+            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + orow * a.N + col0 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              dst[i / 4] = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                       __uint_as_float(v[i + 3]));
+          }
+        } else {
+          // SwiGLU backward, padded row prow, columns i0 .. i0+31 of I:
+          //   dh' = accumulator (dy W_dn), s = sigmoid(g), h = BF16(g s u),
+          //   dh = w dh', dg = dh u s (1 + g (1 - s)), du = dh g s,
+          //   hw = BF16(w h), dw partial += dh' h
+          const int64_t i0 = col0 + c * 32;
+          const __nv_bfloat16 *gu = static_cast<const __nv_bfloat16 *>(a.g_u) + prow * 2 * I;
+          __nv_bfloat16 *dgu = static_cast<__nv_bfloat16 *>(a.d_gu) + prow * 2 * I;
+          __nv_bfloat16 *hwp = static_cast<__nv_bfloat16 *>(a.hw) + prow * I;
+          uint4 gq[4], uq[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            gq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + i0) + q);
+            uq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + I + i0) + q);
+          }
+          const uint32_t *gw = reinterpret_cast<const uint32_t *>(gq);
+          const uint32_t *uw = reinterpret_cast<const uint32_t *>(uq);
+          uint32_t o_dg[16], o_du[16], o_hw[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float dg2[2], du2[2], hw2[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float g = q ? bf16_hi(gw[i]) : bf16_lo(gw[i]);
+              const float u = q ? bf16_hi(uw[i]) : bf16_lo(uw[i]);
+              const float dhp = __uint_as_float(v[2 * i + q]);
+              float sg;
+              const float sl = silu_f(g, sg);
+              const float h = __bfloat162float(__float2bfloat16_rn(sl * u));
+              const float dh = wr * dhp;
+              dg2[q] = dh * u * (sg * (1.0f + g * (1.0f - sg)));
+              du2[q] = dh * sl;
+              hw2[q] = wr * h;
+              dwp = __fmaf_rn(dhp, h, dwp);
+            }
+            o_dg[i] = pack_bf16x2(dg2[0], dg2[1]);
+            o_du[i] = pack_bf16x2(du2[0], du2[1]);
+            o_hw[i] = pack_bf16x2(hw2[0], hw2[1]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            reinterpret_cast<uint4 *>(dgu + i0)[q] =
+                make_uint4(o_dg[4 * q], o_dg[4 * q + 1], o_dg[4 * q + 2], o_dg[4 * q + 3]);
+            reinterpret_cast<uint4 *>(dgu + I + i0)[q] =
+                make_uint4(o_du[4 * q], o_du[4 * q + 1], o_du[4 * q + 2], o_du[4 * q + 3]);
+            reinterpret_cast<uint4 *>(hwp + i0)[q] =
+                make_uint4(o_hw[4 * q], o_hw[4 * q + 1], o_hw[4 * q + 2], o_hw[4 * q + 3]);
+          }
+          if (a.out_f32 != nullptr) {     // dh' itself, for inspection
+            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + prow * a.N + i0);
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              dst[i / 4] = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                       __uint_as_float(v[i + 3]));
+          }
+        }
+      }
+      if (a.epilogue == kBfSwiGLUBwd) a.dw_part[prow * (I / 128) + (col0 / 128)] = dwp;
+    }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
+  if (a.rows_cap <= 0 || a.N % BN != 0) return a.rows_cap <= 0 ? cudaSuccess : cudaErrorInvalidValue;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(k_bf16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
+  }
+  BParams P;
+  P.a = a;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  int64_t tiles;
+  if (a.mode == kBfRows) {
+    if (a.K % BK != 0) return cudaErrorInvalidValue;
+    if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.K, (uint64_t)a.rows_cap, BK, BM, SW))
+      return cudaErrorInvalidValue;
+    if (a.b_mn) {
+      if (!encode_2d_map(&P.tmap_b, BF, 2, a.b, (uint64_t)a.N, (uint64_t)(a.E * a.K), 64, BK, SW))
+        return cudaErrorInvalidValue;
+    } else {
+      if (!encode_2d_map(&P.tmap_b, BF, 2, a.b, (uint64_t)a.K, (uint64_t)(a.E * a.N), BK, BN, SW))
+        return cudaErrorInvalidValue;
+    }
+    tiles = (a.rows_cap / BM) * (a.N / BN);
+  } else {
+    if (a.M % BM != 0) return cudaErrorInvalidValue;
+    if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.M, (uint64_t)a.rows_cap, 64, BK, SW))
+      return cudaErrorInvalidValue;
+    if (!encode_2d_map(&P.tmap_b, BF, 2, a.b, (uint64_t)a.N, (uint64_t)a.rows_cap, 64, BK, SW))
+      return cudaErrorInvalidValue;
+    tiles = (int64_t)a.E * (a.M / BM) * (a.N / BN);
+  }
+  std::memset(&P.tmap_out, 0, sizeof(P.tmap_out));
+  if (a.epilogue == kBfStore && a.out_bf16 != nullptr) {
+    const uint64_t rows = a.mode == kBfRows ? (uint64_t)a.rows_cap : (uint64_t)(a.E * a.M);
+    if (!encode_2d_map(&P.tmap_out, BF, 2, a.out_bf16, (uint64_t)a.N, rows, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
+  int64_t grid = num_sms();
+  if (grid > tiles) grid = tiles;
+  if (grid < 1) grid = 1;
+  k_bf16_gemm<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

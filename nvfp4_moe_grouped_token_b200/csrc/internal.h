@@ -82,6 +82,12 @@ struct PermuteParams {
   // padded end) of each group below rows_cap (scan kernel)
   float *zero_pad_rows = nullptr;
   int64_t rows_cap = 0;
+  // optional: route from router logits [T][E] inside the count kernel; the
+  // chosen ids / weights go to topk_idx_out (which topk_idx must equal) and
+  // topk_w_out
+  const float *logits = nullptr;
+  int32_t *topk_idx_out = nullptr;
+  float *topk_w_out = nullptr;
 };
 int64_t permute_blocks(int64_t T);
 cudaError_t launch_route_count(const PermuteParams &p, cudaStream_t s);
@@ -105,16 +111,80 @@ struct GemmArgs {
   int out_padded;
   float *amax_h;      // SwiGLU: amax of h (per row [rows_cap] or [1])
   int amax_h_rows;
+  // SwiGLU with per-row amax: requantize h inside the launch (nullable = no)
+  uint8_t *req_q;         // [rows_cap][N/4] codes of h
+  uint8_t *req_sf;        // K-step-major scales of h
+  float *req_s_dec;       // [rows_cap]
+  int discard_h;          // drop h's L2 lines once requantized (h undefined after)
+  // plain-store epilogue, non-strict combine: y[t] += w * out_row (FP32
+  // reductions) instead of storing the rows (nullable = store)
+  float *red_y;           // [T][N]
+  const int32_t *red_perm;  // perm[R]: compact sorted row -> t * k + j
+  const float *red_w;       // topk_w [T * k]
+  int red_k;
   int *err;
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
 
+// ---------------------------------------------------------------- BF16 ----
+// BF16 x BF16 -> FP32 grouped GEMM on tcgen05 (kind::f16), for the layer's
+// BF16 backward.
+enum Bf16GemmMode : int {
+  kBfRows = 0,    // per expert e: C[r][n] = sum_k A[r][k] * B_e[n][k], r over e's padded rows
+  kBfWgrad = 1,   // per expert e: C_e[m][n] = sum_{r in group e} A[r][m] * B[r][n]
+};
+enum Bf16Epilogue : int {
+  kBfStore = 0,       // BF16 and/or FP32 output
+  kBfSwiGLUBwd = 1,   // backward of SwiGLU and of the combine's dot (see gemm_bf16.cu)
+};
+
+struct Bf16GemmArgs {
+  int mode = kBfRows;
+  // operand layouts: A is K-major [rows_cap][K] (kBfRows) or MN-major
+  // [rows_cap][M] (kBfWgrad); B is K-major [E][N][K], MN-major [E][K][N]
+  // (kBfRows), or MN-major [rows_cap][N] (kBfWgrad)
+  int b_mn = 0;
+  const void *a = nullptr;
+  const void *b = nullptr;
+  const int32_t *offsets = nullptr, *padded_offsets = nullptr;
+  int E = 1;
+  int64_t rows_cap = 0, M = 0, N = 0, K = 0;
+  int epilogue = kBfStore;
+  void *out_bf16 = nullptr;     // kBfRows: [rows][N] (padded or compact); kBfWgrad: [E][M][N]
+  float *out_f32 = nullptr;
+  int out_padded = 1;
+  // kBfSwiGLUBwd (kBfRows, N = I): the accumulator is dh' = dy_rows W_dn
+  const void *g_u = nullptr;    // BF16 [rows_cap][2I]: gate columns, then up columns
+  const float *w_rows = nullptr;  // [rows_cap] routing weight of each row (0 on padding)
+  void *d_gu = nullptr;         // BF16 [rows_cap][2I] (out)
+  void *hw = nullptr;           // BF16 [rows_cap][I] (out): w * BF16(silu(g) u)
+  float *dw_part = nullptr;     // [rows_cap][I/128] (out): partial <dh', h> per 128 columns
+  int *err = nullptr;
+};
+cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s);
+
+// Backward helpers: gather x and dy rows into the padded grouped layout
+// (zeros on padding rows), the row weights, and ones for the dx combine.
+struct BwdGatherParams {
+  const void *x, *dy;
+  const float *topk_w;
+  const int32_t *topk_idx, *perm, *offsets, *padded_offsets;
+  int64_t T, H, rows_cap;
+  int k, E;
+  void *x_rows, *dy_rows;
+  float *w_rows, *ones;
+};
+cudaError_t launch_bwd_gather(const BwdGatherParams &p, cudaStream_t s);
+cudaError_t launch_bwd_dw(const float *dw_part, int64_t nparts, const int32_t *inv_perm, const int32_t *topk_idx,
+                          const int32_t *offsets, const int32_t *padded_offsets, int64_t T, int k, int E,
+                          float *dw, cudaStream_t s);
+
 cudaError_t launch_combine(const void *d, const int32_t *inv_perm, const float *w, int64_t T, int k,
                            int64_t H, void *y, cudaStream_t s);
+cudaError_t launch_f32_to_bf16(const float *src, int64_t n, void *dst, cudaStream_t s);
 
 cudaError_t launch_wait_selftest(int *err, cudaStream_t s);
-cudaError_t launch_mma_probe(int iters, int n, int sf_a_copies, int sf_b_copies, int mode,
-                             long long *cycles, int *err, const uint8_t *gsrc, int grid, cudaStream_t s);
+cudaError_t launch_mma_peak(int iters, int scale_writes, long long *cycles, int *err, int grid, cudaStream_t s);
 
 int num_sms();
 

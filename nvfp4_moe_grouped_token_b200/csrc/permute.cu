@@ -11,12 +11,16 @@
 //          rank inside its block is the popcount of the masks of the earlier
 //          warps plus that of its own warp below its lane.  Writes the
 //          per-block count of every expert and each (token, slot)'s local rank.
+//          The fused variant starts from router logits: each warp runs the
+//          top-k of its 32 tokens (topk.cuh), writes topk_idx / topk_w and
+//          sets the masks directly -- router and histogram in one pass.
 //   scan   one block: exclusive prefix over blocks per expert (in place), the
 //          expert totals, and their prefix sums -> offsets / padded_offsets.
 //   rank   perm / inv_perm from offsets + block base + local rank (the fused
 //          layer path does this inside the quantize-scatter kernel instead).
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace nvfp4moe {
 
@@ -24,6 +28,9 @@ namespace {
 
 constexpr int kScanThreads = 1024;
 
+// NE == 0: the routing is given (topk_idx); NE > 0: top-k from the router
+// logits first (E <= 32 * NE), written to topk_idx (== p.topk_idx) / topk_w.
+template <int NE>
 __global__ void __launch_bounds__(kRankTokens) k_route_count(const PermuteParams p) {
   extern __shared__ uint32_t smem_u[];
   const int E = p.E, k = p.k;
@@ -34,7 +41,20 @@ __global__ void __launch_bounds__(kRankTokens) k_route_count(const PermuteParams
   const int64_t t = (int64_t)blockIdx.x * kRankTokens + threadIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool live = t < p.T;
-  if (live) {
+  if constexpr (NE > 0) {
+    // warp w: the block's tokens w*32 + i, one at a time; token i is bit i
+    const int64_t t0 = (int64_t)blockIdx.x * kRankTokens + warp * 32;
+    for (int i = 0; i < 32 && t0 + i < p.T; ++i) {
+      int id;
+      float w;
+      warp_topk<NE>(p.logits + (t0 + i) * E, E, k, lane, id, w);
+      if (lane < k) {
+        p.topk_idx_out[(t0 + i) * k + lane] = id;
+        p.topk_w_out[(t0 + i) * k + lane] = w;
+        atomicOr(&masks[warp * E + id], 1u << i);
+      }
+    }
+  } else if (live) {
     const int32_t *row = p.topk_idx + t * k;
     for (int j = 0; j < k; ++j) {
       const int e = __ldg(row + j);
@@ -63,14 +83,15 @@ __global__ void __launch_bounds__(kRankTokens) k_route_count(const PermuteParams
   }
   __syncthreads();
   if (live) {
+    // plain (coherent) loads: the fused variant wrote these ids in this launch
     const int32_t *row = p.topk_idx + t * k;
     const uint32_t below = (1u << lane) - 1u;
     for (int j = 0; j < k; ++j) {
-      const int e = __ldg(row + j);
+      const int e = __ldcg(row + j);
       int32_t r = -1;
       if (e >= 0 && e < E) {
         bool dup = false;
-        for (int jj = 0; jj < j; ++jj) dup |= (__ldg(row + jj) == e);
+        for (int jj = 0; jj < j; ++jj) dup |= (__ldcg(row + jj) == e);
         if (!dup) r = wpre[warp * E + e] + __popc(masks[warp * E + e] & below);
       }
       p.local_rank[t * k + j] = r;
@@ -196,7 +217,17 @@ cudaError_t launch_route_count(const PermuteParams &p, cudaStream_t s) {
   const int64_t nblk = permute_blocks(p.T);
   if (nblk == 0) return cudaSuccess;
   const size_t smem = (size_t)8 * p.E * sizeof(uint32_t);
-  k_route_count<<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+  if (p.logits == nullptr) {
+    k_route_count<0><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+  } else {
+    if (p.topk_idx != p.topk_idx_out || p.k > p.E || p.k > 32) return cudaErrorInvalidValue;
+    if (p.E <= 32) k_route_count<1><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+    else if (p.E <= 64) k_route_count<2><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+    else if (p.E <= 128) k_route_count<4><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+    else if (p.E <= 256) k_route_count<8><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+    else if (p.E <= 512) k_route_count<16><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+    else k_route_count<32><<<(unsigned)nblk, kRankTokens, smem, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -11,24 +11,17 @@
 // over the chosen k.  The choice compares the FP32 logits exactly, so it is
 // bit-reproducible; only the weights carry rounding (expf and one division).
 //
-// One warp per token: lane l holds logits l, l+32, ...; each of the k rounds
-// is a warp arg-best under the strict order (larger logit, then lower id),
-// so every lane agrees on the winner whatever the reduction order.
-#include <climits>
-
+// One warp per token (warp_topk in topk.cuh).  The fused variant that also
+// builds the routing histogram lives in permute.cu.
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace nvfp4moe {
 
 namespace {
 
 constexpr int kRouteWarps = 8;
-
-// (va, ia) ranks before (vb, ib): larger logit first, then lower expert id
-__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
-}
 
 template <int NE>   // logits per lane: E <= 32 * NE
 __global__ void __launch_bounds__(kRouteWarps * 32)
@@ -37,54 +30,12 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   if (t >= T) return;
-  const float *row = logits + t * E;
-  float v[NE];
-  uint32_t taken = 0;   // bit i: expert i*32 + lane already chosen (or beyond E)
-#pragma unroll
-  for (int i = 0; i < NE; ++i) {
-    const int e = i * 32 + lane;
-    v[i] = e < E ? __ldg(row + e) : 0.0f;
-    if (e >= E) taken |= 1u << i;
-  }
-  int my_id = 0;        // slot `lane` for lane < k
-  float my_v = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    float bv = 0.0f;
-    int bi = INT_MAX;   // INT_MAX: this lane has nothing left
-#pragma unroll
-    for (int i = 0; i < NE; ++i) {
-      const int e = i * 32 + lane;
-      if (!((taken >> i) & 1u) && (bi == INT_MAX || ranks_before(v[i], e, bv, bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != INT_MAX && (bi == INT_MAX || ranks_before(ov, oi, bv, bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    // k <= E, so a winner exists; its owner marks it taken
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == j) {
-      my_id = bi;
-      my_v = bv;
-    }
-  }
-  // weights: exp(l_j - l_max) over the chosen, normalised; the sum is a fixed
-  // butterfly, so the result does not depend on anything but the logits
-  const float m = __shfl_sync(0xffffffffu, my_v, 0);
-  const float z = lane < k ? expf(my_v - m) : 0.0f;
-  float s = z;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  int my_id;
+  float my_w;
+  warp_topk<NE>(logits + t * E, E, k, lane, my_id, my_w);
   if (lane < k) {
     idx_out[t * k + lane] = my_id;
-    w_out[t * k + lane] = __fdiv_rn(z, s);
+    w_out[t * k + lane] = my_w;
   }
 }
 

@@ -29,6 +29,10 @@ STRICT = 0x2
 SF_MMA_LAYOUT = 0x4
 OUT_PADDED = 0x8
 W_GATE_UP = 0x10
+KEEP_H = 0x20
+BWD_KEEP_DH = 0x40
+FAST_COMBINE = 0x80
+FUSED_REQUANT = 0x100
 
 _vp, _i64, _i32, _u32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_size_t
 
@@ -48,6 +52,9 @@ _SIGS = {
     "moe_permute": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_route_topk": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "moe_route_permute": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_layer_from_logits": (_i32, [_vp, _vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights), _i64,
+                                            _i64, _i64, _i32, _i32, _vp, _vp, _vp, _u32, _vp, _sz, _vp]),
     "moe_quantize_permute": (_i32, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _i64, _u32, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64,
@@ -64,7 +71,12 @@ _SIGS = {
                                          _vp, _u32, _vp, _sz, _vp, ctypes.POINTER(_vp)]),
     "nvfp4moe_encode_e2m1": (_i32, [_vp, _i64, _vp, _vp]),
     "nvfp4moe_encode_ue4m3": (_i32, [_vp, _i64, _vp, _vp]),
-    "nvfp4moe_mma_probe": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "nvfp4moe_mma_peak": (_i32, [_i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_expert_layer_backward_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32, _u32]),
+    "moe_expert_layer_backward_workspace_offsets": (_i32, [_i64, _i64, _i64, _i32, _i32, _u32,
+                                                           ctypes.POINTER(_i64)]),
+    "moe_expert_layer_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp,
+                                         _vp, _vp, _vp, _vp, _u32, _vp, _sz, _vp]),
     "nvfp4moe_num_sms": (_i32, []),
 }
 
@@ -159,6 +171,18 @@ def moe_route_topk(logits, k, topk_idx, topk_w, stream=None):
     T, E = logits.shape
     _check(lib().moe_route_topk(_p(logits), T, E, k, _p(topk_idx), _p(topk_w), _stream(stream)),
            "moe_route_topk")
+
+
+def moe_route_permute(logits, k, topk_idx, topk_w, offsets, padded_offsets, perm, inv_perm, workspace,
+                      stream=None):
+    """moe_route_permute: router top-k fused with the routing histogram, then
+    the permutation; workspace of moe_permute_workspace_size(T, k, E)."""
+    _dev(logits, topk_idx, topk_w, offsets, padded_offsets, perm, inv_perm, workspace)
+    T, E = logits.shape
+    _check(lib().moe_route_permute(_p(logits), T, E, k, _p(topk_idx), _p(topk_w), _p(offsets),
+                                   _p(padded_offsets), _p(perm), _p(inv_perm), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "moe_route_permute")
 
 
 def moe_permute_noalloc(topk_idx, E, offsets, padded_offsets, perm, inv_perm, stream=None):
@@ -266,6 +290,21 @@ def moe_expert_layer(x, topk_idx, topk_w, w_gate_up: NVFP4Weights, w_down: NVFP4
            "moe_expert_layer")
 
 
+def moe_expert_layer_from_logits(x, logits, w_gate_up: NVFP4Weights, w_down: NVFP4Weights, topk_idx, topk_w,
+                                 y, workspace, flags=0, stream=None):
+    """moe_expert_layer_from_logits: the layer routed from router logits
+    inside its histogram kernel; topk_idx / topk_w are written."""
+    _dev(x, logits, topk_idx, topk_w, y, workspace)
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    I = w_down.K
+    gu, dn = w_gate_up.struct(), w_down.struct()
+    _check(lib().moe_expert_layer_from_logits(_p(x), _p(logits), ctypes.byref(gu), ctypes.byref(dn), T, H, I,
+                                              w_down.E, k, _p(topk_idx), _p(topk_w), _p(y), flags, _p(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(stream)),
+           "moe_expert_layer_from_logits")
+
+
 STAGES = ["route", "quantize_permute", "gate_up_swiglu", "requant_h", "down", "combine"]
 
 
@@ -287,6 +326,73 @@ def moe_expert_layer_profiled(x, topk_idx, topk_w, w_gate_up: NVFP4Weights, w_do
                                            _stream(stream), arr), "moe_expert_layer_profiled")
 
 
+# ------------------------------------------------------------- backward --
+
+def moe_expert_layer_backward_workspace_size(T, H, I, E, k, flags=0) -> int:
+    return int(lib().moe_expert_layer_backward_workspace_size(T, H, I, E, k, flags))
+
+
+_BWD_REGIONS = ["err", "offsets", "padded_offsets", "perm", "inv_perm", "x_rows", "dy_rows", "w_rows", "g",
+                "dg", "hw", "dw_part", "dx_rows", "dh"]
+
+
+def moe_expert_layer_backward_workspace_offsets(T, H, I, E, k, flags=0) -> dict:
+    arr = (ctypes.c_int64 * 16)()
+    _check(lib().moe_expert_layer_backward_workspace_offsets(T, H, I, E, k, flags, arr),
+           "moe_expert_layer_backward_workspace_offsets")
+    out = {name: int(arr[i]) for i, name in enumerate(_BWD_REGIONS)}
+    out["rows_cap"] = int(arr[14])
+    out["total"] = int(arr[15])
+    return out
+
+
+def moe_expert_layer_backward(x, topk_idx, topk_w, w_gate_up, w_down, dy, dx, d_topk_w, workspace,
+                              dw_gate_up_bf16=None, dw_gate_up_f32=None, dw_down_bf16=None, dw_down_f32=None,
+                              flags=0, stream=None):
+    """Backward of the layer in the BF16-backward mode (moe_expert_layer_backward):
+    w_gate_up [E][2I][H] and w_down [E][H][I] are the BF16 weights."""
+    _dev(x, topk_idx, topk_w, w_gate_up, w_down, dy, dx, d_topk_w, workspace, dw_gate_up_bf16, dw_gate_up_f32,
+         dw_down_bf16, dw_down_f32)
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    E, N2, _ = w_gate_up.shape
+    _check(lib().moe_expert_layer_backward(_p(x), _p(topk_idx), _p(topk_w), _p(w_gate_up), _p(w_down), _p(dy), T,
+                                           H, N2 // 2, E, k, _p(dx), _p(d_topk_w), _p(dw_gate_up_bf16),
+                                           _p(dw_gate_up_f32), _p(dw_down_bf16), _p(dw_down_f32), flags,
+                                           _p(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "moe_expert_layer_backward")
+
+
+def backward_views(workspace: torch.Tensor, T, H, I, E, k, flags=0) -> dict:
+    """Typed views of the backward workspace's regions (for inspection in tests)."""
+    o = moe_expert_layer_backward_workspace_offsets(T, H, I, E, k, flags)
+    cap = o["rows_cap"]
+    R = T * k
+    ws = workspace
+
+    def view(name, nbytes, dtype, shape):
+        return ws[o[name]:o[name] + nbytes].view(dtype).view(*shape)
+
+    v = {
+        "rows_cap": cap,
+        "offsets": view("offsets", (E + 1) * 4, torch.int32, (E + 1,)),
+        "padded_offsets": view("padded_offsets", (E + 1) * 4, torch.int32, (E + 1,)),
+        "perm": view("perm", R * 4, torch.int32, (R,)),
+        "inv_perm": view("inv_perm", R * 4, torch.int32, (T, k)),
+        "x_rows": view("x_rows", cap * H * 2, torch.bfloat16, (cap, H)),
+        "dy_rows": view("dy_rows", cap * H * 2, torch.bfloat16, (cap, H)),
+        "w_rows": view("w_rows", cap * 4, torch.float32, (cap,)),
+        "g": view("g", cap * 2 * I * 2, torch.bfloat16, (cap, 2 * I)),
+        "dg": view("dg", cap * 2 * I * 2, torch.bfloat16, (cap, 2 * I)),
+        "hw": view("hw", cap * I * 2, torch.bfloat16, (cap, I)),
+        "dw_part": view("dw_part", cap * (I // 128) * 4, torch.float32, (cap, I // 128)),
+        "dx_rows": view("dx_rows", R * H * 2, torch.bfloat16, (R, H)),
+    }
+    if flags & BWD_KEEP_DH:
+        v["dh"] = view("dh", cap * I * 4, torch.float32, (cap, I))
+    return v
+
+
 def nvfp4moe_encode_e2m1(y: torch.Tensor, codes: torch.Tensor, stream=None):
     _dev(y, codes)
     _check(lib().nvfp4moe_encode_e2m1(_p(y), y.numel(), _p(codes), _stream(stream)), "encode_e2m1")
@@ -297,28 +403,27 @@ def nvfp4moe_encode_ue4m3(v: torch.Tensor, codes: torch.Tensor, stream=None):
     _check(lib().nvfp4moe_encode_ue4m3(_p(v), v.numel(), _p(codes), _stream(stream)), "encode_ue4m3")
 
 
-def mma_probe(iters: int, n: int = 256, sf_a_copies: int = 4, sf_b_copies: int = 8, mode: int = 0,
-              grid: int = 0, stream=None) -> dict:
-    """nvfp4moe_mma_probe: dense block-scaled FP4 MMA throughput on this GPU.
-    Returns TFLOP/s (from CUDA events) and FLOP per SM per cycle."""
+def mma_peak(iters: int = 4000, scale_writes: bool = True, grid: int = 0, stream=None) -> dict:
+    """nvfp4moe_mma_peak: dense block-scaled FP4 MMA throughput on this GPU,
+    timed with CUDA events on the launching stream.  Returns TFLOP/s and FLOP
+    per SM per cycle."""
     grid = grid or lib().nvfp4moe_num_sms()
     cyc = torch.zeros(grid, dtype=torch.int64, device="cuda")
-    ws = torch.zeros(256 + 55296, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     s = torch.cuda.current_stream() if stream is None else stream
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s)
-    _check(lib().nvfp4moe_mma_probe(iters, n, sf_a_copies, sf_b_copies, mode, grid, _p(cyc), _p(ws),
-                                    _stream(stream)), "nvfp4moe_mma_probe")
+    _check(lib().nvfp4moe_mma_peak(iters, 1 if scale_writes else 0, grid, _p(cyc), _p(ws), _stream(s)),
+           "nvfp4moe_mma_peak")
     e1.record(s)
     torch.cuda.synchronize()
     if device_status(ws) != OK:
-        raise NVFP4Error("mma probe wait timed out")
-    flop = grid * iters * 4 * 2.0 * 128 * n * 64
+        raise NVFP4Error("mma peak probe wait timed out")
+    flop = grid * iters * 4 * 2.0 * 128 * 256 * 64
     ms = e0.elapsed_time(e1)
     c = cyc.float().mean().item()
     return {"tflops": flop / (ms * 1e-3) / 1e12, "flop_per_sm_cycle": flop / grid / c, "ms": ms,
-            "cycles_mean": c, "grid": grid, "n": n, "sf_a_copies": sf_a_copies, "sf_b_copies": sf_b_copies,
-            "mode": mode}
+            "cycles_mean": c, "grid": grid, "iters": iters, "scale_writes": bool(scale_writes)}
 
 
 # ------------------------------------------------------------------ helpers --

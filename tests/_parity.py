@@ -1,5 +1,9 @@
 """Comparison helpers shared by the GPU parity tests.
 
+The reference values come from the plain C++ oracle (oracle/nvfp4_oracle.cpp
+through oracle.cpp); index helpers (padded row positions, the expert of a
+sorted row, BF16 spacing) are plain numpy here.
+
 Tolerances (benchmark spec of the problem):
   * codes, scales, amax, S_dec, offsets and permutation: bit-exact;
   * a GEMM output in FP32: |gpu - exact| <= 1e-5 * sum_k |a_k w_k| + 1e-6;
@@ -12,7 +16,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from oracle import moe, nvfp4
+from oracle import cpp
 
 REL = 1e-5
 ABS = 1e-6
@@ -31,16 +35,63 @@ def check_f32(gpu: np.ndarray, exact: np.ndarray, sum_abs: np.ndarray, what: str
     return float((err / np.maximum(sum_abs, 1e-30)).max())
 
 
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of BF16 numbers at |v| (8 significant bits; fixed below 2^-126)."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    _, e2 = np.frexp(np.where(a > 0, a, 1.0))
+    e = np.where(a > 0, e2 - 1, -126)
+    return np.exp2(np.maximum(e, -126) - 7.0)
+
+
+# elements accepted only through the second branch of check_bf16, per check
+RELAXED_COUNTS = {}
+
+
 def check_bf16(gpu: np.ndarray, exact: np.ndarray, extra_bound: np.ndarray, what: str):
     """gpu: float32 values of BF16 results; exact: fp64 reference before
-    rounding; extra_bound: propagated FP32 error bound of the GPU's value."""
+    rounding; extra_bound: propagated FP32 error bound of the GPU's value.
+
+    An element passes when it is within one BF16 ulp of the exact value
+    rounded to BF16, or -- the second branch -- when the FP32 bound itself
+    spans more than that (outputs near cancellation).  The second branch's
+    count is recorded (RELAXED_COUNTS), printed, and must stay a tiny share."""
     gpu = gpu.astype(np.float64)
-    ref = nvfp4.round_to_bf16(exact).astype(np.float64)
-    ulp = nvfp4.bf16_ulp(ref)
+    ref = cpp.round_to_bf16(exact).astype(np.float64)
+    ulp = bf16_ulp(ref)
     d = np.abs(gpu - ref)
-    ok = (d <= ulp) | (np.abs(gpu - exact) <= extra_bound + 0.5 * nvfp4.bf16_ulp(gpu))
+    first = d <= ulp
+    second = np.abs(gpu - exact) <= extra_bound + 0.5 * bf16_ulp(gpu)
+    ok = first | second
     assert ok.all(), (f"{what}: {int((~ok).sum())} of {ok.size} BF16 values off; "
                       f"worst |d|/ulp {float((d / ulp).max()):.3g}")
+    relaxed = int((~first).sum())
+    RELAXED_COUNTS[what] = RELAXED_COUNTS.get(what, 0) + relaxed
+    print(f"{what}: {ok.size} BF16 values, {relaxed} within the FP32 bound only")
+    assert relaxed <= max(4, 1e-3 * ok.size), f"{what}: {relaxed} values pass only through the FP32 bound"
+    return relaxed
+
+
+def padded_rows(perm_info) -> np.ndarray:
+    """Padded row index of every sorted row r (length R)."""
+    off = perm_info["offsets"].astype(np.int64)
+    pad = perm_info["padded_offsets"].astype(np.int64)
+    E = len(off) - 1
+    expert_of_r = np.repeat(np.arange(E), np.diff(off))
+    r = np.arange(off[-1])
+    return r - off[expert_of_r] + pad[expert_of_r]
+
+
+def expert_of_rows(offsets: np.ndarray) -> np.ndarray:
+    off = np.asarray(offsets, dtype=np.int64)
+    return np.repeat(np.arange(len(off) - 1), np.diff(off))
+
+
+def unpack_nibbles(q: np.ndarray) -> np.ndarray:
+    q = np.asarray(q, dtype=np.uint8)
+    out = np.empty(q.shape[:-1] + (q.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = q & 0xF
+    out[..., 1::2] = q >> 4
+    return out
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -71,7 +122,7 @@ def check_weights_exact(prep, w_cpu: torch.Tensor, gate_up: bool, experts=None):
     sf = prep.sf.cpu()
     s_dec = prep.s_dec.cpu().numpy()
     for e in (range(E) if experts is None else experts):
-        r = nvfp4.quantize(w_cpu[e].float().numpy(), per_token=False)
+        r = cpp.quantize(w_cpu[e].float().numpy(), per_token=False)
         qe = q[e]
         sfe = ops_rowmajor_expert(sf, e, N, K)
         if gate_up:
@@ -96,12 +147,12 @@ def dequant_weights(prep, e: int, gate_up: bool) -> np.ndarray:
     if gate_up:
         q = undo_gate_up_interleave(q, N)
         sf = undo_gate_up_interleave(sf, N)
-    return nvfp4.dequantize(q, sf, prep.s_dec[e:e + 1].cpu().numpy())
+    return cpp.dequantize(q, sf, prep.s_dec[e:e + 1].cpu().numpy())
 
 
 def swiglu_bound(g, u, tg, tu):
     """Bound on |silu(g')u' - silu(g)u| for |g'-g| <= tg, |u'-u| <= tu
     (|silu'| <= 1.1), plus FP32 epilogue rounding (a few ulps of h)."""
-    s = np.abs(moe.silu(g))
+    s = np.abs(g / (1.0 + np.exp(-np.asarray(g, dtype=np.float64))))
     h = np.abs(s * u)
     return 1.1 * tg * (np.abs(u) + tu) + (s + 1.1 * tg) * tu + 8 * 2.0 ** -24 * h + 1e-30

@@ -24,12 +24,40 @@ def test_layer_flops_closed_form():
 
 def test_stage_bytes_count_each_tensor_once():
     cfg = workloads.CONFIGS["moe30b"]
-    b = bench.stage_bytes(cfg, 0)
     R, H, I, E = 131072, 2048, 768, 128
     nv = 0.5625
-    assert b["combine"] == R * H * 2 + 16384 * H * 2 + R * 8
-    assert b["down"] == R * I * nv + E * H * I * nv + R * H * 2
-    assert b["requant_h"] == R * I * (2 + nv)
+    # separate requantization: h leaves gate_up in BF16 and a second pass requantizes it
+    for per_tensor in (False, True):
+        b = bench.stage_bytes(cfg, per_tensor=per_tensor)
+        assert b["combine"] == R * H * 2 + 16384 * H * 2 + R * 8
+        assert b["down"] == R * I * nv + E * H * I * nv + R * H * 2
+        assert b["gate_up_swiglu"] == R * H * nv + E * 2 * I * H * nv + R * I * 2
+        assert b["requant_h"] == R * I * (2 + nv)
+    # fused into gate_up (per-token only): the GEMM writes h's codes, no requant stage
+    b = bench.stage_bytes(cfg, per_tensor=False, fused_requant=True)
+    assert b["gate_up_swiglu"] == R * H * nv + E * 2 * I * H * nv + R * I * nv
+    assert "requant_h" not in b
+    # the whole step moves about 2 GB at the moe30b shape (the survey's figure)
+    total = sum(bench.stage_bytes(cfg, per_tensor=False, fused_requant=True).values())
+    assert 1.6e9 < total < 2.1e9
+
+
+def test_kernel_rooflines_fractions_follow_from_the_times():
+    cfg = workloads.CONFIGS["moe30b"]
+    stage_ms = {"route": 0.02, "quantize_permute": 0.05, "gate_up_swiglu": 0.2, "down": 0.15, "combine": 0.1}
+    pk = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}
+    fp4 = {"mma_only": 8000.0, "with_scale_writes": 7500.0}
+    rows = {r["stage"]: r for r in bench.kernel_rooflines(cfg, stage_ms, False, pk, fp4, None)}
+    fl = bench.layer_flops(cfg)
+    sb = bench.stage_bytes(cfg, False)
+    gu = rows["gate_up_swiglu"]
+    assert abs(gu["tflops"] - fl["gate_up"] / 0.2e-3 / 1e12) < 1e-6
+    assert abs(gu["frac_fp4_peak"] - gu["tflops"] / 8000.0) < 1e-12
+    assert rows["route"]["bound"] == "latency"
+    for name in ("quantize_permute", "down", "combine"):
+        r = rows[name]
+        assert abs(r["gbs"] - sb[name] / (stage_ms[name] * 1e-3) / 1e9) < 1e-6
+        assert abs(r["frac_hbm"] - r["gbs"] / 6500.0) < 1e-12
 
 
 def test_job_throughput_is_all_tokens_over_slowest_rank():

@@ -5,10 +5,11 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import moe, nvfp4
+from oracle import cpp
 from nvfp4_moe_grouped_token_b200 import ops, workloads
 
-from _parity import (check_bf16, check_f32, check_weights_exact, dequant_weights, gemm_bound)
+from _parity import (check_bf16, check_f32, check_weights_exact, dequant_weights, expert_of_rows, gemm_bound,
+                     padded_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,9 +48,9 @@ class Problem:
         ops.moe_quantize_permute(x.cuda(), idx.cuda(), self.inv, self.off, self.pad, E, self.q,
                                  self.sf, self.sdec, self.cap, flags=flags, amax_out=amax)
         torch.cuda.synchronize()
-        self.info = moe.permutation(idx.numpy(), E)
-        self.qx = nvfp4.quantize(x.float().numpy(), per_token)
-        self.prow = moe.padded_rows(self.info)
+        self.info = cpp.permutation(idx.numpy(), E)
+        self.qx = cpp.quantize(x.float().numpy(), per_token)
+        self.prow = padded_rows(self.info)
         self.tok = self.info["perm"] // k
 
     def check_activation_rows(self, rows=None):
@@ -76,16 +77,15 @@ class Problem:
 
     def reference(self, rows):
         """fp64 GEMM and sum|aw| for the given sorted rows."""
-        xh = nvfp4.dequantize(self.qx["q"], self.qx["sf"], self.qx["s_dec"])
-        e_of = moe.expert_of_rows(self.info["offsets"])[rows]
+        xh = cpp.dequantize(self.qx["q"], self.qx["sf"], self.qx["s_dec"])
+        e_of = expert_of_rows(self.info["offsets"])[rows]
         a = xh[self.tok[rows]]
         exact = np.empty((len(rows), self.N))
         sabs = np.empty_like(exact)
         for e in np.unique(e_of):
             m = e_of == e
             we = dequant_weights(self.prep, int(e), gate_up=False)
-            exact[m] = a[m] @ we.T
-            sabs[m] = np.abs(a[m]) @ np.abs(we).T
+            exact[m], sabs[m] = cpp.gemm_rows(a[m], we, with_abs=True)
         return exact, sabs
 
     def check_outputs(self, rows=None, padded=False):

@@ -5,11 +5,11 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import moe, nvfp4
+from oracle import cpp
 from nvfp4_moe_grouped_token_b200 import ops, workloads
 
-from _parity import (check_bf16, check_weights_exact, dequant_weights, gemm_bound,
-                     swiglu_bound)
+from _parity import (bf16_ulp, check_bf16, check_weights_exact, dequant_weights, expert_of_rows, gemm_bound,
+                     padded_rows, swiglu_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,8 +30,11 @@ class Layer:
         self.idx = self.inp["topk_idx"].cuda()
         self.w = self.inp["topk_w"].cuda()
 
-    def run(self):
-        ops.moe_expert_layer(self.x, self.idx, self.w, self.wgu, self.wdn, self.y, self.ws, self.flags)
+    def run(self, keep_h=True):
+        # KEEP_H leaves h readable for the stage-by-stage checks; the outputs
+        # do not depend on it (test_keep_h_does_not_change_outputs)
+        flags = self.flags | (ops.KEEP_H if keep_h else 0)
+        ops.moe_expert_layer(self.x, self.idx, self.w, self.wgu, self.wdn, self.y, self.ws, flags)
         assert ops.device_status(self.ws) == 0
         c = self.cfg
         self.v = ops.layer_views(self.ws, c.T, c.H, c.I, c.E, c.k, self.flags)
@@ -46,13 +49,13 @@ class Layer:
             check_weights_exact(self.wgu, self.inp["w_gate_up"], True, experts=range(min(E, 3)))
             check_weights_exact(self.wdn, self.inp["w_down"], False, experts=range(min(E, 3)))
         # 1-2. permutation (exact, all rows)
-        info = moe.permutation(idx, E)
+        info = cpp.permutation(idx, E)
         for key in ("offsets", "padded_offsets", "perm"):
             assert np.array_equal(v[key].cpu().numpy(), info[key]), key
         assert np.array_equal(v["inv_perm"].cpu().numpy(), info["inv_perm"])
-        prow = moe.padded_rows(info)
+        prow = padded_rows(info)
         tok = info["perm"] // k
-        e_of = moe.expert_of_rows(info["offsets"])
+        e_of = expert_of_rows(info["offsets"])
         # rows under test
         if sample_tokens is None:
             rows = np.arange(T * k)
@@ -63,7 +66,7 @@ class Layer:
         pr = prow[rows]
         cap = v["rows_cap"]
         # 3. x quantized once per token, scattered (exact)
-        qx = nvfp4.quantize(x, self.per_token)
+        qx = cpp.quantize(x, self.per_token)
         xq = v["x_q"].cpu().numpy()
         xsf = ops.sf_kstep_to_rowmajor(v["x_sf"].cpu(), cap, H).numpy()
         assert np.array_equal(xq[pr], qx["q"][tok[rows]])
@@ -71,7 +74,7 @@ class Layer:
         sd_want = qx["s_dec"][tok[rows]] if self.per_token else np.full(len(rows), qx["s_dec"][0])
         assert np.array_equal(v["x_sdec"].cpu().numpy()[pr], sd_want)
         # 4. gate_up + SwiGLU -> h (tolerance, teacher-forced from the exact codes)
-        xh = nvfp4.dequantize(qx["q"], qx["sf"], qx["s_dec"])
+        xh = cpp.dequantize(qx["q"], qx["sf"], qx["s_dec"])
         a = xh[tok[rows]]
         g = np.empty((len(rows), 2 * I))
         gs = np.empty_like(g)
@@ -82,18 +85,17 @@ class Layer:
         for e in np.unique(e_of[rows]):
             m = e_of[rows] == e
             we = dequant_weights(self.wgu, int(e), gate_up=True)
-            g[m] = a[m] @ we.T
-            gs[m] = np.abs(a[m]) @ np.abs(we).T
-        h_exact = moe.swiglu(g, I)
+            g[m], gs[m] = cpp.gemm_rows(a[m], we, with_abs=True)
+        h_exact = cpp.swiglu(g, I)
         tg, tu = gemm_bound(gs[:, :I]), gemm_bound(gs[:, I:])
         check_bf16(h_gpu, h_exact, swiglu_bound(g[:, :I], g[:, I:], tg, tu), "h")
         # 5. requant of the GPU's h, amax reused from the epilogue (exact)
         if self.per_token:
-            qh = nvfp4.quantize(h_gpu, True)
+            qh = cpp.quantize(h_gpu, True)
         else:
             valid_h = h_gpu_all[prow]                     # every routed row
             amax = np.abs(valid_h).max()
-            qh = nvfp4.quantize(h_gpu, False, amax_in=np.array([amax], np.float32))
+            qh = cpp.quantize(h_gpu, False, amax_in=np.array([amax], np.float32))
         hq = v["h_q"].cpu().numpy()
         hsf = ops.sf_kstep_to_rowmajor(v["h_sf"].cpu(), cap, I).numpy()
         assert np.array_equal(hq[pr], qh["q"])
@@ -101,12 +103,11 @@ class Layer:
         hsd = v["h_sdec"].cpu().numpy()[pr]
         assert np.array_equal(hsd, qh["s_dec"] if self.per_token else np.full(len(rows), qh["s_dec"][0]))
         # 6. down GEMM from the GPU's h codes -> D (tolerance)
-        hh = nvfp4.dequantize(qh["q"], qh["sf"], qh["s_dec"])
+        hh = cpp.dequantize(qh["q"], qh["sf"], qh["s_dec"])
         for e in np.unique(e_of[rows]):
             m = e_of[rows] == e
             we = dequant_weights(self.wdn, int(e), gate_up=False)
-            d_exact[m] = hh[m] @ we.T
-            d_abs[m] = np.abs(hh[m]) @ np.abs(we).T
+            d_exact[m], d_abs[m] = cpp.gemm_rows(hh[m], we, with_abs=True)
         d_gpu = v["d"].float().cpu().numpy()[rows]
         check_bf16(d_gpu, d_exact, gemm_bound(d_abs), "D")
         # 7. combine from the GPU's D (fp32 sum of k terms vs fp64: one BF16 ulp)
@@ -124,7 +125,7 @@ class Layer:
 SMALL = workloads.LayerConfig("small", T=300, H=256, I=256, E=8, k=2, seed=21)
 
 
-@pytest.mark.parametrize("flags", [0, ops.SCALE_PER_TOKEN, ops.STRICT])
+@pytest.mark.parametrize("flags", [0, ops.SCALE_PER_TOKEN, ops.STRICT, ops.STRICT | ops.FUSED_REQUANT])
 def test_small_layer_all_rows(flags):
     L = Layer(SMALL, flags)
     L.run()
@@ -135,14 +136,65 @@ def test_small_layer_end_to_end_against_full_oracle():
     L = Layer(SMALL, ops.STRICT)
     L.run()
     x = L.inp["x"].float().numpy()
-    wgu = moe.QuantWeights(L.inp["w_gate_up"].float().numpy())
-    wdn = moe.QuantWeights(L.inp["w_down"].float().numpy())
-    ref = moe.expert_layer(x, L.inp["topk_idx"].numpy(), L.inp["topk_w"].numpy(), wgu, wdn, per_token=True)
+    ref = cpp.expert_layer(x, L.inp["topk_idx"].numpy(), L.inp["topk_w"].numpy(),
+                           L.inp["w_gate_up"].float().numpy(), L.inp["w_down"].float().numpy(), per_token=True)
     y = L.y.float().cpu().numpy()
     rel = np.linalg.norm(y - ref["y"]) / np.linalg.norm(ref["y"])
     # not teacher-forced: requant code flips near rounding boundaries are expected
     print(f"end-to-end relative L2 difference vs oracle: {rel:.3g}")
     assert rel < 2e-2
+
+
+@pytest.mark.parametrize("cfg_name", ["small", "moe30b", "dense4b"])
+def test_fused_requant_matches_the_separate_pass(cfg_name):
+    """NVFP4MOE_FUSED_REQUANT requantizes h inside the gate_up GEMM (m-tile-
+    major tile order, worker warps); without KEEP_H it also drops h's cache
+    lines.  Codes, scales, S_dec, D and y must be bitwise those of the
+    separate requantization pass, and h itself with KEEP_H."""
+    cfg = {"small": SMALL, "moe30b": workloads.CONFIGS["moe30b"], "dense4b": workloads.CONFIGS["dense4b"]}[cfg_name]
+    L = Layer(cfg, ops.STRICT)
+    L.run(keep_h=True)
+    keys = ("h_q", "h_sf", "h_sdec", "d", "h_amax", "h")
+    ref = {key: L.v[key].clone() for key in keys}
+    y_ref = L.y.clone()
+    for extra in (ops.FUSED_REQUANT | ops.KEEP_H, ops.FUSED_REQUANT):
+        L.ws.zero_()
+        L.y.zero_()
+        L.flags = ops.STRICT | extra
+        L.run(keep_h=False)
+        for key in keys:
+            if key == "h" and not extra & ops.KEEP_H:
+                continue
+            assert torch.equal(L.v[key].view(torch.uint8), ref[key].view(torch.uint8)), (key, extra)
+        assert torch.equal(L.y.view(torch.int16), y_ref.view(torch.int16)), extra
+
+
+@pytest.mark.parametrize("cfg_name", ["small", "moe30b"])
+def test_fast_combine_matches_the_ordered_sum(cfg_name):
+    """NVFP4MOE_FAST_COMBINE (non-strict): the down GEMM adds w * D (FP32)
+    straight into y's FP32 accumulator.  Against the ordered path's BF16 D:
+    |y_fast - sum_j w_j D_j| <= sum_j |w_j| ulp(D_j)/2 (D's BF16 rounding the
+    fast path skips) + the FP32 sum's error + half a BF16 ulp of y."""
+    cfg = SMALL if cfg_name == "small" else workloads.CONFIGS["moe30b"]
+    L = Layer(cfg, ops.SCALE_PER_TOKEN)
+    L.run()
+    d = L.v["d"].float().cpu().numpy().astype(np.float64)
+    inv = L.v["inv_perm"].cpu().numpy()
+    wts = L.inp["topk_w"].numpy().astype(np.float64)
+    ref = np.zeros((cfg.T, cfg.H))
+    slack = np.zeros_like(ref)
+    for j in range(cfg.k):
+        dj = d[inv[:, j]]
+        ref += wts[:, j:j + 1] * dj
+        slack += np.abs(wts[:, j:j + 1]) * (0.5 * bf16_ulp(dj) + cfg.k * 2.0 ** -23 * np.abs(dj))
+    ops.moe_expert_layer(L.x, L.idx, L.w, L.wgu, L.wdn, L.y, L.ws, ops.SCALE_PER_TOKEN | ops.FAST_COMBINE)
+    assert ops.device_status(L.ws) == 0
+    y = L.y.float().cpu().numpy().astype(np.float64)
+    err = np.abs(y - ref)
+    bound = slack + 0.5 * bf16_ulp(y) + 1e-30
+    assert np.all(err <= bound), float((err / bound).max())
+    with pytest.raises(ops.NVFP4Error):
+        ops.moe_expert_layer(L.x, L.idx, L.w, L.wgu, L.wdn, L.y, L.ws, ops.STRICT | ops.FAST_COMBINE)
 
 
 def test_moe30b_layer_sampled():

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import moe
+from oracle import cpp
 from nvfp4_moe_grouped_token_b200 import ops, workloads
 
 pytestmark = pytest.mark.gpu
@@ -27,7 +27,7 @@ def _gpu_permute(idx_cpu, E):
 def _check(idx_cpu, E):
     off, pad, perm, inv, st = _gpu_permute(idx_cpu, E)
     assert st == 0
-    r = moe.permutation(idx_cpu.numpy(), E)
+    r = cpp.permutation(idx_cpu.numpy(), E)
     assert np.array_equal(off, r["offsets"])
     assert np.array_equal(pad, r["padded_offsets"])
     assert np.array_equal(perm, r["perm"])

@@ -1,9 +1,11 @@
-"""GPU quantizer and codec parity: bit-exact against the CPU oracle."""
+"""GPU quantizer and codec parity: bit-exact against the C++ CPU oracle,
+including exhaustive sweeps of the hardware E2M1 / UE4M3 conversions over
+every finite binary32 bit pattern."""
 import numpy as np
 import pytest
 import torch
 
-from oracle import nvfp4
+from oracle import cpp
 from nvfp4_moe_grouped_token_b200 import ops
 
 from _parity import sf_rowmajor
@@ -51,7 +53,7 @@ SHAPES = [(1, 64), (5, 64), (37, 256), (300, 768), (129, 2048), (64, 2560), (100
 def test_quantize_bit_exact(M, K, per_token):
     x = _x(M, K, seed=M * 7 + K)
     q, sf, s_dec, amax = _gpu_quant(x, per_token)
-    r = nvfp4.quantize(x.float().numpy(), per_token)
+    r = cpp.quantize(x.float().numpy(), per_token)
     assert np.array_equal(amax, r["amax"])
     assert np.array_equal(s_dec, r["s_dec"])
     assert np.array_equal(sf, r["sf"])
@@ -63,20 +65,20 @@ def test_quantize_bit_exact(M, K, per_token):
 def test_quantize_hard_inputs(kind, per_token):
     x = _x(200, 512, seed=3, kind=kind)
     q, sf, s_dec, amax = _gpu_quant(x, per_token)
-    r = nvfp4.quantize(x.float().numpy(), per_token)
+    r = cpp.quantize(x.float().numpy(), per_token)
     assert np.array_equal(s_dec, r["s_dec"]) and np.array_equal(sf, r["sf"]) and np.array_equal(q, r["q"])
 
 
 @pytest.mark.parametrize("per_token", [False, True])
 def test_quantize_mma_layout_and_amax_reuse(per_token):
     x = _x(333, 1024, seed=5)
-    ref = nvfp4.quantize(x.float().numpy(), per_token)
+    ref = cpp.quantize(x.float().numpy(), per_token)
     q, sf, s_dec, amax = _gpu_quant(x, per_token, sf_mma=True)
     assert np.array_equal(sf, ref["sf"]) and np.array_equal(q, ref["q"])
     # amax reuse: the given amax is used as is (here: twice the true one)
     a2 = ref["amax"] * np.float32(2)
     q2, sf2, s2, amax2 = _gpu_quant(x, per_token, amax_in=a2)
-    r2 = nvfp4.quantize(x.float().numpy(), per_token, amax_in=a2)
+    r2 = cpp.quantize(x.float().numpy(), per_token, amax_in=a2)
     assert np.array_equal(amax2, a2)
     assert np.array_equal(q2, r2["q"]) and np.array_equal(sf2, r2["sf"]) and np.array_equal(s2, r2["s_dec"])
 
@@ -91,7 +93,7 @@ def _neighbourhoods(points, span=64):
 
 
 def test_e2m1_hardware_rounding_matches_definition():
-    g = nvfp4.E2M1_MAGNITUDES
+    g = cpp.e2m1_decode(np.arange(8))
     mids = (g[1:] + g[:-1]) / 2
     pts = np.concatenate([g, mids, [6.5, 7.0, 100.0, 1e-30, 2.0 ** -126]])
     y = _neighbourhoods(pts[pts > 0])
@@ -102,13 +104,13 @@ def test_e2m1_hardware_rounding_matches_definition():
     codes = torch.empty(y.size, dtype=torch.uint8, device="cuda")
     ops.nvfp4moe_encode_e2m1(torch.from_numpy(y).cuda(), codes)
     got = codes.cpu().numpy()
-    want = nvfp4.e2m1_encode(y)
+    want = cpp.e2m1_encode(y)
     bad = got != want
     assert not bad.any(), list(zip(y[bad][:8], got[bad][:8], want[bad][:8]))
 
 
 def test_ue4m3_hardware_rounding_matches_definition():
-    g = nvfp4.UE4M3_VALUES
+    g = cpp.ue4m3_decode(np.arange(127))
     mids = (g[1:] + g[:-1]) / 2
     pts = np.concatenate([g[1:], mids, [448.0, 464.0, 480.0, 1e4, 2.0 ** -10]])
     v = _neighbourhoods(pts)
@@ -118,9 +120,44 @@ def test_ue4m3_hardware_rounding_matches_definition():
     codes = torch.empty(v.size, dtype=torch.uint8, device="cuda")
     ops.nvfp4moe_encode_ue4m3(torch.from_numpy(v).cuda(), codes)
     got = codes.cpu().numpy()
-    want = nvfp4.ue4m3_encode(v)
+    want = cpp.ue4m3_encode(v)
     bad = got != want
     assert not bad.any(), list(zip(v[bad][:8], got[bad][:8], want[bad][:8]))
+
+
+CHUNK = 1 << 26
+
+
+def _sweep(lo, hi, encode_gpu, encode_cpu):
+    """GPU codes of every binary32 pattern in [lo, hi) against the oracle's,
+    chunk by chunk (the oracle builds its inputs from the same bit range)."""
+    for start in range(lo, hi, CHUNK):
+        n = min(CHUNK, hi - start)
+        bits = torch.arange(start, start + n, dtype=torch.int64, device="cuda")
+        vals = (bits - (1 << 32) * (bits >= (1 << 31))).to(torch.int32).view(torch.float32)
+        codes = torch.empty(n, dtype=torch.uint8, device="cuda")
+        encode_gpu(vals, codes)
+        got = codes.cpu().numpy()
+        want = encode_cpu(start, n)
+        if not np.array_equal(got, want):
+            bad = np.nonzero(got != want)[0][:8]
+            raise AssertionError([(hex(start + int(i)), int(got[i]), int(want[i])) for i in bad])
+        del bits, vals, codes
+
+
+def test_e2m1_exhaustive_all_finite_fp32():
+    """cvt.rn.satfinite.e2m1x2.f32 on all 2^32 - 2^24 finite patterns (both
+    signs) equals the definition (round to nearest even, saturate at 6, sign
+    kept on -0)."""
+    _sweep(0, 0x7F800000, ops.nvfp4moe_encode_e2m1, cpp.e2m1_encode_bits)
+    _sweep(0x80000000, 0xFF800000, ops.nvfp4moe_encode_e2m1, cpp.e2m1_encode_bits)
+
+
+def test_ue4m3_exhaustive_all_nonnegative_finite_fp32():
+    """cvt.rn.satfinite.e4m3x2.f32 on every non-negative finite pattern (the
+    quantizer only converts non-negative block scales) equals UE4M3 round to
+    nearest even saturating at 448."""
+    _sweep(0, 0x7F800000, ops.nvfp4moe_encode_ue4m3, cpp.ue4m3_encode_bits)
 
 
 def test_empty_is_noop():

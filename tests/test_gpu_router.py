@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import moe
+from oracle import cpp
 from nvfp4_moe_grouped_token_b200 import ops
 
 pytestmark = pytest.mark.gpu
@@ -37,7 +37,7 @@ def _route_gpu(lg, k):
 
 def _check(lg, k):
     idx, w = _route_gpu(lg, k)
-    ref_idx, ref_w = moe.route_topk(lg.numpy(), k)
+    ref_idx, ref_w = cpp.route_topk(lg.numpy(), k)
     assert np.array_equal(idx, ref_idx)
     err = np.abs(w.astype(np.float64) - ref_w)
     assert np.all(err <= W_RTOL * ref_w + 1e-38), float((err / ref_w).max())
@@ -78,8 +78,8 @@ def test_routed_tokens_permute_like_the_oracle():
     ws = torch.zeros(ops.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
     ops.moe_permute(idx, E, off, pad, perm, inv, ws)
     assert ops.device_status(ws) == 0
-    ref_idx, _ = moe.route_topk(lg.numpy(), k)
-    info = moe.permutation(ref_idx, E)
+    ref_idx, _ = cpp.route_topk(lg.numpy(), k)
+    info = cpp.permutation(ref_idx, E)
     assert np.array_equal(off.cpu().numpy(), info["offsets"])
     assert np.array_equal(perm.cpu().numpy(), info["perm"])
     assert np.array_equal(inv.cpu().numpy(), info["inv_perm"])
@@ -96,3 +96,64 @@ def test_routed_tokens_permute_like_the_oracle():
     us = e0.elapsed_time(e1) / 20 * 1e3
     print(f"moe_route_topk T={T} E={E} k={k}: {us:.1f} us per call "
           f"({T * E * 4 / (us * 1e-6) / 1e9:.0f} GB/s of logits)")
+
+
+def _route_permute(lg, k):
+    T, E = lg.shape
+    idx = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    pad = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(ops.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
+    ops.moe_route_permute(lg.cuda(), k, idx, w, off, pad, perm, inv, ws)
+    assert ops.device_status(ws) == 0
+    return [t.cpu().numpy() for t in (idx, w, off, pad, perm, inv)]
+
+
+@pytest.mark.parametrize("T,E,k", [(16384, 128, 8), (1000, 16, 4), (333, 1000, 32), (257, 33, 1), (130, 256, 8)])
+def test_fused_route_permute_matches_oracle(T, E, k):
+    """Router top-k folded into the routing-histogram kernel: ids and the
+    whole permutation bit-exact against the oracle's router + permutation,
+    weights within the router tolerance and bitwise equal to the standalone
+    router kernel's (the same arithmetic)."""
+    lg = _logits(T, E, seed=T + E + k, ties=(E == 128))
+    idx, w, off, pad, perm, inv = _route_permute(lg, k)
+    ref_idx, ref_w = cpp.route_topk(lg.numpy(), k)
+    assert np.array_equal(idx, ref_idx)
+    assert np.all(np.abs(w.astype(np.float64) - ref_w) <= W_RTOL * ref_w + 1e-38)
+    idx2, w2 = _route_gpu(lg, k)
+    assert np.array_equal(w.view(np.int32), w2.view(np.int32))
+    info = cpp.permutation(ref_idx, E)
+    for name, got in (("offsets", off), ("padded_offsets", pad), ("perm", perm), ("inv_perm", inv)):
+        assert np.array_equal(got, info[name]), name
+
+
+def test_layer_from_logits_equals_layer_with_routed_inputs():
+    """moe_expert_layer_from_logits routes inside the layer's histogram
+    kernel; its output is bitwise that of moe_expert_layer fed the same
+    routing (which the standalone router produces)."""
+    from nvfp4_moe_grouped_token_b200 import workloads
+    cfg = workloads.LayerConfig("logits_layer", T=2000, H=512, I=256, E=16, k=4, seed=31)
+    inp = workloads.layer_inputs(cfg)
+    lg = _logits(cfg.T, cfg.E, seed=3).cuda()
+    wgu = ops.nvfp4_prepare_weights(inp["w_gate_up"].cuda(), gate_up=True)
+    wdn = ops.nvfp4_prepare_weights(inp["w_down"].cuda(), gate_up=False)
+    x = inp["x"].cuda()
+    for flags in (ops.STRICT, 0):
+        ws = torch.zeros(ops.moe_expert_layer_workspace_size(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, flags),
+                         dtype=torch.uint8, device="cuda")
+        idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+        w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+        y1 = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+        ops.moe_expert_layer_from_logits(x, lg, wgu, wdn, idx, w, y1, ws, flags)
+        assert ops.device_status(ws) == 0
+        idx2 = torch.empty_like(idx)
+        w2 = torch.empty_like(w)
+        ops.moe_route_topk(lg, cfg.k, idx2, w2)
+        assert torch.equal(idx, idx2) and torch.equal(w.view(torch.int32), w2.view(torch.int32))
+        y2 = torch.empty_like(y1)
+        ops.moe_expert_layer(x, idx2, w2, wgu, wdn, y2, ws, flags)
+        assert ops.device_status(ws) == 0
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), flags
