@@ -19,11 +19,18 @@ done in IEEE binary32 with round-to-nearest-even, one operation at a time,
 exactly as the quantizer on the GPU must do it; everything else (dequantize,
 GEMM, SwiGLU, combine) is fp64.
 
+The oracle the GPU tests compare against is the plain C++ one
+(nvfp4_oracle.cpp, built with g++ -O2 -ffp-contract=off -fno-fast-math and
+bound by ``cpp``).  The numpy modules are a second, separately written opinion
+that the CPU tests check against it bit for bit.
+
 Modules
+  cpp      -- ctypes binding of the C++ oracle (codecs, quantize, routing,
+              permutation, grouped GEMM, SwiGLU, combine, layer, backward)
   nvfp4    -- E2M1 / UE4M3 codecs, BF16 rounding, quantize, dequantize
   moe      -- routing, permutation, grouped GEMM, SwiGLU + requantize, combine,
               the layer
   backward -- the layer's gradients in the BF16-backward mode
   mxfp8    -- MXFP8 (E4M3 elements, E8M0 block scales) for the W4A8 variant
 """
-from . import nvfp4, moe, backward, mxfp8  # noqa: F401
+from . import nvfp4, moe, backward, mxfp8, cpp  # noqa: F401

@@ -1,9 +1,9 @@
 """Backward of the MoE expert layer -- CPU oracle (test infrastructure only).
 
-Source passage: news.hamidun.com "miniTE ... 1.39x over BF16 on
-Qwen3-30B-A3B", the speed table: besides the full NVFP4 path the pages time a
-mode that runs the forward in NVFP4 and the backward in BF16 (about 1.33-1.37x
-over BF16).  The pages give no formulas for it.
+Source passage: www.aib.vote "miniTE report, NVFP4 RL stability",
+paragraph 1: besides the full NVFP4 path the report times a mode that runs the
+forward in NVFP4 and the backward in BF16 (about 1.33-1.37x over BF16 for the
+full training update on 8xB300).  The pages give no formulas for it.
 
 Reading taken where the pages are silent:
   R16  BF16-backward mode: the backward is the exact gradient of the layer
