@@ -62,6 +62,8 @@ _SIGS = {
     "orc_swiglu_backward": (None, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "orc_expert_layer_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _vp, _vp,
                                          _vp, _vp]),
+    "orc_expert_layer_w4a16": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
+                                      ctypes.POINTER(_LayerOut)]),
     "orc_expert_layer": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32,
                                 ctypes.POINTER(_LayerOut)]),
 }
@@ -317,3 +319,29 @@ def expert_layer_backward(x, topk_idx, topk_w, w_gate_up, w_down, dy) -> dict:
     if rc != 0:
         raise ValueError("orc_expert_layer_backward: bad routing entry")
     return out
+
+
+def expert_layer_w4a16(x, topk_idx, topk_w, w_gate_up, w_down) -> dict:
+    """R19: the layer with BF16 activations and NVFP4 weights (x not
+    quantized, h not requantized).  Returns y, offsets, perm, inv_perm, h
+    (BF16, sorted rows) and d."""
+    x = _c(x, np.float32)
+    idx = _c(topk_idx, np.int32)
+    tw = _c(topk_w, np.float32)
+    wgu = _c(w_gate_up, np.float32)
+    wdn = _c(w_down, np.float32)
+    T, H = x.shape
+    k = idx.shape[1]
+    E, N2, _ = wgu.shape
+    I = N2 // 2
+    R = T * k
+    o = {"y": np.empty((T, H), np.float32), "offsets": np.empty(E + 1, np.int32),
+         "padded_offsets": np.empty(E + 1, np.int32), "perm": np.empty(R, np.int32),
+         "inv_perm": np.empty((T, k), np.int32), "h": np.empty((R, I), np.float32), "d": np.empty((R, H), np.float32)}
+    fields = {name: arr.ctypes.data for name, arr in o.items()}
+    st = _LayerOut(**fields)
+    rc = lib().orc_expert_layer_w4a16(_p(x), _p(idx), _p(tw), _p(wgu), _p(wdn), T, H, I, E, k, threads(),
+                                      ctypes.byref(st))
+    if rc != 0:
+        raise ValueError("orc_expert_layer_w4a16: bad shape or routing entry")
+    return o

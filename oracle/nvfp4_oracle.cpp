@@ -42,6 +42,11 @@
 //       slot order.
 //   R15 top-k routing: the k largest logits (ties to the lower expert id),
 //       slots in descending order, weights = softmax over the chosen k.
+//   R19 W4A16 variant (www.aib.vote "miniTE report, NVFP4 RL stability",
+//       paragraph 3 measures W4A16 beside W4A8 and W4A4 without formulas):
+//       the same NVFP4 weights, BF16 activations: x is not quantized and h is
+//       not requantized; G = x W_gu^T on the dequantized weights in fp64,
+//       h = BF16(silu(g) u), D = BF16(h W_dn^T), then the same combine.
 //   R16 backward, BF16-backward mode (www.aib.vote "miniTE report, NVFP4 RL
 //       stability", paragraph 1 times "NVFP4 forward, BF16 backward" without
 //       formulas): the exact gradient of the unquantized layer on its BF16
@@ -473,6 +478,52 @@ int orc_expert_layer(const float *x, const int32_t *topk_idx, const float *topk_
   put(out->h_q, hq);
   put(out->h_sf, hsf);
   put(out->h_s_dec, hsd);
+  put(out->d, d);
+  return 0;
+}
+
+// R19: the W4A16 variant of orc_expert_layer -- BF16 activations, NVFP4
+// weights.  Outputs y, the permutation, h (BF16, sorted rows) and D.
+int orc_expert_layer_w4a16(const float *x, const int32_t *topk_idx, const float *topk_w, const float *w_gate_up,
+                           const float *w_down, int64_t T, int64_t H, int64_t I, int E, int k, int threads,
+                           OrcLayerOut *out) {
+  if (H % 16 != 0 || I % 16 != 0 || out == nullptr || out->y == nullptr) return -1;
+  const int64_t R = T * k;
+  std::vector<int32_t> off(E + 1), pad(E + 1), perm(R), inv(R);
+  if (orc_permutation(topk_idx, T, k, E, off.data(), pad.data(), perm.data(), inv.data()) != 0) return -1;
+  std::vector<double> a(R * H);
+  for (int64_t p = 0; p < R; ++p) {
+    const int64_t t = perm[p] / k;
+    for (int64_t c = 0; c < H; ++c) a[p * H + c] = x[t * H + c];
+  }
+  std::vector<double> wgu((int64_t)E * 2 * I * H), wdn((int64_t)E * H * I);
+  for (int e = 0; e < E; ++e) {
+    std::vector<uint8_t> q(2 * I * H / 2), sc(2 * I * H / 16);
+    float sd, am;
+    orc_quantize(w_gate_up + (int64_t)e * 2 * I * H, 2 * I, H, 0, nullptr, q.data(), sc.data(), &sd, &am);
+    orc_dequantize(q.data(), sc.data(), &sd, 2 * I, H, 0, &wgu[(int64_t)e * 2 * I * H]);
+    std::vector<uint8_t> q2(H * I / 2), s2(H * I / 16);
+    orc_quantize(w_down + (int64_t)e * H * I, H, I, 0, nullptr, q2.data(), s2.data(), &sd, &am);
+    orc_dequantize(q2.data(), s2.data(), &sd, H, I, 0, &wdn[(int64_t)e * H * I]);
+  }
+  std::vector<double> gu(R * 2 * I), hd(R * I), hb(R * I), dd(R * H);
+  orc_grouped_gemm(a.data(), off.data(), E, wgu.data(), 2 * I, H, gu.data(), nullptr, threads);
+  orc_swiglu(gu.data(), R, I, hd.data());
+  std::vector<float> h(R * I);
+  orc_round_bf16_n(hd.data(), R * I, h.data());
+  for (int64_t i = 0; i < R * I; ++i) hb[i] = h[i];
+  orc_grouped_gemm(hb.data(), off.data(), E, wdn.data(), H, I, dd.data(), nullptr, threads);
+  std::vector<float> d(R * H);
+  orc_round_bf16_n(dd.data(), R * H, d.data());
+  orc_combine(d.data(), H, inv.data(), topk_w, T, k, out->y);
+  auto put = [](auto *dst, const auto &src) {
+    if (dst != nullptr) std::copy(src.begin(), src.end(), dst);
+  };
+  put(out->offsets, off);
+  put(out->padded_offsets, pad);
+  put(out->perm, perm);
+  put(out->inv_perm, inv);
+  put(out->h, h);
   put(out->d, d);
   return 0;
 }

@@ -332,3 +332,39 @@ def test_swiglu_backward_closed_form():
         assert dgu[0, 3 + i] == pytest.approx(dh * gg * s, rel=1e-14, abs=1e-300)
         assert h[0, i] == pytest.approx(gg * s * u, rel=1e-14, abs=1e-300)
     assert dgu[0, 0] == 0.5 * 1.0 * 5.0 * 0.5     # silu'(0) = 1/2
+
+
+def test_w4a16_layer_against_per_token_brute_force():
+    """R19 (BF16 activations, NVFP4 weights): the oracle's permuted grouped
+    path against a per-(token, slot) brute force with exactly rounded dot
+    products, and against the W4A4 layer's weight quantization (the same
+    dequantized weights)."""
+    rng = np.random.default_rng(61)
+    T, H, I, E, k = 12, 64, 48, 6, 2
+    x = nvfp4.round_to_bf16(rng.standard_normal((T, H)))
+    idx = np.stack([rng.choice(5, k, replace=False) for _ in range(T)]).astype(np.int32)   # expert 5 empty
+    tw = rng.random((T, k)).astype(np.float32)
+    w_gu = nvfp4.round_to_bf16(rng.standard_normal((E, 2 * I, H)) * 0.05)
+    w_dn = nvfp4.round_to_bf16(rng.standard_normal((E, H, I)) * 0.05)
+    out = cpp.expert_layer_w4a16(x, idx, tw, w_gu, w_dn)
+
+    def wq(w):
+        q = cpp.quantize(w, False)
+        return cpp.dequantize(q["q"], q["sf"], q["s_dec"])
+
+    wgu = [wq(w_gu[e]) for e in range(E)]
+    wdn = [wq(w_dn[e]) for e in range(E)]
+    y = np.zeros((T, H), np.float32)
+    for t in range(T):
+        acc = np.zeros(H)
+        for j in range(k):
+            e = int(idx[t, j])
+            g = np.array([math.fsum(x[t].astype(np.float64) * wgu[e][n]) for n in range(2 * I)])
+            h = nvfp4.round_to_bf16(g[:I] / (1.0 + np.exp(-g[:I])) * g[I:]).astype(np.float64)
+            pos = int(out["inv_perm"][t, j])
+            assert np.array_equal(out["h"][pos], h.astype(np.float32)), (t, j)
+            d = nvfp4.round_to_bf16(np.array([math.fsum(h * wdn[e][n]) for n in range(H)]))
+            assert np.array_equal(out["d"][pos], d), (t, j)
+            acc = acc + float(tw[t, j]) * d.astype(np.float64)
+        y[t] = nvfp4.round_to_bf16(acc)
+    assert np.array_equal(out["y"], y)
