@@ -405,6 +405,42 @@ int moe_expert_layer_backward(const void *x, const int32_t *topk_idx,
                               void *workspace, size_t workspace_bytes,
                               nvfp4moe_stream_t stream);
 
+/* --------------------------------------------------------------- W4A16 -- */
+/* The MoE expert layer with BF16 activations and NVFP4 weights.  The
+ * miniTE report on NVFP4 RL stability (www.aib.vote, paragraph 3) measures
+ * this variant beside W4A8 and W4A4 and gives no formulas; this reads it as
+ * the W4A4 layer without the activation quantizers:
+ *   G = x_rows W_gu,e^T,  h = BF16(silu(g) * u),  D = BF16(h W_dn,e^T),
+ *   y[t] = BF16(sum_j topk_w[t][j] * D[t][j])  (slot order, FP32),
+ * with W the dequantized NVFP4 weights (codes x block scale x S_dec).  The
+ * weights stay 4-bit in memory; each K-step of a weight tile is converted to
+ * BF16 in shared memory and multiplied on the tensor cores (tcgen05
+ * kind::f16, FP32 accumulation); S_dec is applied to the accumulator.
+ *   x, topk_idx, topk_w, y, T, H, I, E, k   as for moe_expert_layer
+ *   w_gate_up, w_down   prepared exactly as for moe_expert_layer
+ *   flags      0 (reserved)
+ *   workspace  moe_expert_layer_w4a16_workspace_size() bytes
+ * Requirements: those of moe_expert_layer.  Errors: those of
+ * moe_expert_layer; the device error word (nvfp4moe_device_status) reports
+ * a bounded wait that gave up. */
+size_t moe_expert_layer_w4a16_workspace_size(int64_t T, int64_t H, int64_t I,
+                                             int E, int k, uint32_t flags);
+/* Byte offsets of the W4A16 workspace's regions: [0] error word, [1] offsets,
+ * [2] padded_offsets, [3] perm, [4] inv_perm, [5] x rows (BF16, padded
+ * grouped layout, zero padding rows), [6] h (BF16 [rows_cap][I]), [7] D
+ * (BF16, compact sorted rows), [8..13] 0, [14] rows_cap (a count), [15] total
+ * bytes.  `out` must hold 16 int64 (host memory). */
+int moe_expert_layer_w4a16_workspace_offsets(int64_t T, int64_t H, int64_t I,
+                                             int E, int k, uint32_t flags,
+                                             int64_t *out);
+int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx,
+                           const float *topk_w,
+                           const nvfp4moe_weights *w_gate_up,
+                           const nvfp4moe_weights *w_down, int64_t T,
+                           int64_t H, int64_t I, int E, int k, void *y,
+                           uint32_t flags, void *workspace,
+                           size_t workspace_bytes, nvfp4moe_stream_t stream);
+
 /* ---------------------------------------------------------- diagnostics -- */
 /* The hardware conversions the quantizer uses, exposed so their rounding can
  * be checked against the format definition: codes[i] = E2M1_rne_satfinite(y[i])

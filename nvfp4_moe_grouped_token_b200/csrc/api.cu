@@ -141,6 +141,31 @@ BwdLayout bwd_layout(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t fla
   return L;
 }
 
+// Workspace of the W4A16 layer: [0] header, [1] offsets, [2] padded offsets,
+// [3] perm, [4] inv_perm, [5] x rows (padded), [6] h (padded), [7] D
+// (compact), [14] rows_cap, [15] total bytes.
+BwdLayout w4a16_layout(int64_t T, int64_t H, int64_t I, int E, int k) {
+  const int64_t R = T * k;
+  const int64_t cap = layer_rows_cap(T, k, E);
+  Carve c;
+  BwdLayout L;
+  for (int i = 0; i < 16; ++i) L.v[i] = 0;
+  L.v[0] = c.take(kHeaderBytes);
+  L.v[1] = c.take((E + 1) * 4);
+  L.v[2] = c.take((E + 1) * 4);
+  L.v[3] = c.take(R * 4);
+  L.v[4] = c.take(R * 4);
+  L.v[5] = c.take(cap * H * 2);
+  L.v[6] = c.take(cap * I * 2);
+  L.v[7] = c.take(R * H * 2);
+  L.counts = c.take(permute_blocks(T) * E * 4);
+  L.local_rank = c.take(R * 4);
+  L.ones = 0;
+  L.v[14] = cap;
+  L.v[15] = c.off;
+  return L;
+}
+
 bool per_token(uint32_t flags) { return (flags & (NVFP4MOE_SCALE_PER_TOKEN | NVFP4MOE_STRICT)) != 0; }
 
 int check_weights(const nvfp4moe_weights *w, int64_t E, int64_t N, int64_t K) {
@@ -870,6 +895,120 @@ int nvfp4moe_encode_e2m1(const float *y, int64_t n, uint8_t *codes, nvfp4moe_str
 int nvfp4moe_encode_ue4m3(const float *v, int64_t n, uint8_t *codes, nvfp4moe_stream_t stream) {
   if (n < 0 || (n > 0 && (v == nullptr || codes == nullptr))) return NVFP4MOE_ERR_INVALID_ARG;
   return cuda_rc(launch_encode_ue4m3(v, n, codes, st(stream)));
+}
+
+
+// ------------------------------------------------------------------ W4A16 --
+
+size_t moe_expert_layer_w4a16_workspace_size(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
+  (void)flags;
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+  return (size_t)w4a16_layout(T, H, I, E, k).v[15];
+}
+
+int moe_expert_layer_w4a16_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags,
+                                             int64_t *out) {
+  (void)flags;
+  if (out == nullptr || T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  const BwdLayout L = w4a16_layout(T, H, I, E, k);
+  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
+  return NVFP4MOE_OK;
+}
+
+int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *topk_w,
+                           const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down, int64_t T, int64_t H,
+                           int64_t I, int E, int k, void *y, uint32_t flags, void *workspace, size_t workspace_bytes,
+                           nvfp4moe_stream_t stream) {
+  if (T < 0 || H <= 0 || I <= 0 || k < 1 || k > 32 || E < 1 || flags != 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || H % 256 != 0 || I % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_weights(w_gate_up, E, 2 * I, H);
+  if (rc != NVFP4MOE_OK) return rc;
+  if (!(w_gate_up->flags & NVFP4MOE_W_GATE_UP)) return NVFP4MOE_ERR_INVALID_ARG;
+  rc = check_weights(w_down, E, H, I);
+  if (rc != NVFP4MOE_OK) return rc;
+  if (T == 0) return NVFP4MOE_OK;
+  if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || y == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  const BwdLayout L = w4a16_layout(T, H, I, E, k);
+  if (workspace == nullptr || (int64_t)workspace_bytes < L.v[15]) return NVFP4MOE_ERR_WORKSPACE;
+  const int64_t cap = L.v[14];
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int *err = reinterpret_cast<int *>(ws + L.v[0]);
+  int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.v[1]);
+  int32_t *padded = reinterpret_cast<int32_t *>(ws + L.v[2]);
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.v[3]);
+  int32_t *inv_perm = reinterpret_cast<int32_t *>(ws + L.v[4]);
+  void *x_rows = ws + L.v[5];
+  void *h = ws + L.v[6];
+  void *d = ws + L.v[7];
+  NVFP4MOE_TRY(cudaMemsetAsync(ws + L.v[0], 0, kHeaderBytes, s));
+
+  // routing metadata, then the rows of x in the padded grouped layout
+  PermuteParams pp;
+  pp.topk_idx = topk_idx;
+  pp.T = T;
+  pp.k = k;
+  pp.E = E;
+  pp.block_counts = reinterpret_cast<int32_t *>(ws + L.counts);
+  pp.local_rank = reinterpret_cast<int32_t *>(ws + L.local_rank);
+  pp.offsets = offsets;
+  pp.padded_offsets = padded;
+  pp.perm = perm;
+  pp.inv_perm = inv_perm;
+  pp.err = err;
+  NVFP4MOE_TRY(launch_route_count(pp, s));
+  NVFP4MOE_TRY(launch_route_scan(pp, s));
+  NVFP4MOE_TRY(launch_route_rank(pp, s));
+  BwdGatherParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.x = x;
+  gp.topk_w = topk_w;
+  gp.topk_idx = topk_idx;
+  gp.perm = perm;
+  gp.offsets = offsets;
+  gp.padded_offsets = padded;
+  gp.T = T;
+  gp.H = H;
+  gp.rows_cap = cap;
+  gp.k = k;
+  gp.E = E;
+  gp.x_rows = x_rows;
+  NVFP4MOE_TRY(launch_bwd_gather(gp, s));
+
+  Bf16GemmArgs base;
+  base.mode = kBfRows;
+  base.offsets = offsets;
+  base.padded_offsets = padded;
+  base.E = E;
+  base.rows_cap = cap;
+  base.err = err;
+  // gate_up with NVFP4 weights, SwiGLU epilogue -> h (padded rows)
+  Bf16GemmArgs g1 = base;
+  g1.a = x_rows;
+  g1.b = w_gate_up->q;
+  g1.b_sf = w_gate_up->sf;
+  g1.s_dec_w = w_gate_up->s_dec;
+  g1.N = 2 * I;
+  g1.K = H;
+  g1.epilogue = kBfSwiGLUFwd;
+  g1.out_bf16 = h;
+  g1.out_padded = 1;
+  NVFP4MOE_TRY(launch_bf16_gemm(g1, s));
+  // down with NVFP4 weights -> D (compact sorted rows)
+  Bf16GemmArgs g2 = base;
+  g2.a = h;
+  g2.b = w_down->q;
+  g2.b_sf = w_down->sf;
+  g2.s_dec_w = w_down->s_dec;
+  g2.N = H;
+  g2.K = I;
+  g2.epilogue = kBfStore;
+  g2.out_bf16 = d;
+  g2.out_padded = 0;
+  NVFP4MOE_TRY(launch_bf16_gemm(g2, s));
+  NVFP4MOE_TRY(launch_combine(d, inv_perm, topk_w, T, k, H, y, s));
+  return NVFP4MOE_OK;
 }
 
 }  // extern "C"

@@ -29,12 +29,15 @@ __device__ __forceinline__ int find_group_dev(const int32_t *padded, int E, int6
 // One warp per padded row p < padded_offsets[E]: the row's token t (from the
 // permutation) gives x_rows[p] = x[t], dy_rows[p] = dy[t], w_rows[p] =
 // topk_w[t][j]; padding rows get zeros.  ones[r] = 1 for every routed row.
+// dy / dy_rows, w_rows and ones are optional (the W4A16 forward gathers x
+// alone).
 __global__ void __launch_bounds__(kGatherWarps * 32) k_bwd_gather(const BwdGatherParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
   const int64_t R = p.T * p.k;
-  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R; r += (int64_t)gridDim.x * blockDim.x)
-    p.ones[r] = 1.0f;
+  if (p.ones != nullptr)
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R; r += (int64_t)gridDim.x * blockDim.x)
+      p.ones[r] = 1.0f;
   int64_t used = __ldg(p.padded_offsets + p.E);
   if (used > p.rows_cap) used = p.rows_cap;
   if (row >= used) return;
@@ -52,22 +55,15 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_bwd_gather(const BwdGathe
   }
   const int64_t hv = p.H >> 3;   // uint4 per row
   uint4 *xo = static_cast<uint4 *>(p.x_rows) + row * hv;
-  uint4 *dyo = static_cast<uint4 *>(p.dy_rows) + row * hv;
-  if (t >= 0) {
-    const uint4 *xs = static_cast<const uint4 *>(p.x) + t * hv;
-    const uint4 *dys = static_cast<const uint4 *>(p.dy) + t * hv;
-    for (int64_t c = lane; c < hv; c += 32) {
-      xo[c] = __ldg(xs + c);
-      dyo[c] = __ldg(dys + c);
-    }
-  } else {
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int64_t c = lane; c < hv; c += 32) {
-      xo[c] = z;
-      dyo[c] = z;
-    }
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  const uint4 *xs = static_cast<const uint4 *>(p.x) + (t >= 0 ? t : 0) * hv;
+  for (int64_t c = lane; c < hv; c += 32) xo[c] = t >= 0 ? __ldg(xs + c) : z;
+  if (p.dy_rows != nullptr) {
+    uint4 *dyo = static_cast<uint4 *>(p.dy_rows) + row * hv;
+    const uint4 *dys = static_cast<const uint4 *>(p.dy) + (t >= 0 ? t : 0) * hv;
+    for (int64_t c = lane; c < hv; c += 32) dyo[c] = t >= 0 ? __ldg(dys + c) : z;
   }
-  if (lane == 0) p.w_rows[row] = w;
+  if (lane == 0 && p.w_rows != nullptr) p.w_rows[row] = w;
 }
 
 // dw[t][j] = sum over the row's partials (I/128 of them, in column order) of

@@ -445,10 +445,394 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// W4A16: BF16 activations x NVFP4 weights.  The weights stay 4-bit in HBM
+// (codes + UE4M3 block scales, the layout the W4A4 GEMM reads); converter
+// warps turn each K-step's weight tile into BF16 in shared memory, in the
+// 128-byte-swizzled K-major layout a TMA load would have produced, and the
+// MMAs are the kind::f16 ones above.  code x block scale is exact in BF16
+// (at most 2 + 4 significant bits, exponents well inside the range), so the
+// converted operand is exactly the dequantized weight divided by the
+// per-expert S_dec, which the epilogue applies to the FP32 accumulator.
+//
+//   raw ring (4 stages): A 16 KB (TMA, swizzled) + codes 8 KB (TMA, 256 rows
+//     x 32 bytes, unswizzled) + scales 1 KB (two 512-byte atoms, bulk copies)
+//   converted ring (2 slots): B as BF16, 32 KB each
+//   warp 0: producer; warp 1: TMEM owner + MMA issuer; warps 2-9: epilogue
+//   (two per TMEM lane quarter); warps 10-17: converters, four rows' halves
+//   per lane and K-step.
+namespace w4 {
+constexpr int RS = 4;
+constexpr int CS = 2;
+constexpr int kCodesBytes = BN * BK / 2;                  // 8 KB
+constexpr int kSfBytes = BN * BK / 16;                    // 1 KB
+constexpr int kRawBytes = kABytes + kCodesBytes + kSfBytes;
+constexpr int kThreads = 576;
+constexpr int kEpiWarp0 = 2, kConvWarp0 = 10, kConvWarps = 8;
+constexpr size_t kConvOff = (size_t)RS * kRawBytes;
+constexpr size_t kStagingOff = kConvOff + (size_t)CS * kBBytes;
+constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
+constexpr size_t kSmemBytes = kBarrierOff + 256 + 1024;
+static_assert(kRawBytes % 1024 == 0 && kBBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kConvWarps * 32 * 2 == 2 * BN, "each converter lane covers two half rows");
+}  // namespace w4
+
+// Eight E2M1 codes (one word; element 2b is the low nibble of byte b) ->
+// four BF16 pairs in element order.  The 3-bit magnitude indexes two
+// eight-entry byte tables held in registers (the high and the low byte of the
+// BF16 value of 0, 0.5, 1, 1.5, 2, 3, 4, 6); the code's sign bit becomes
+// bit 15 or 31 of its pair.
+__device__ __forceinline__ void e2m1x8_to_bf16x2(uint32_t c, uint32_t (&w)[4]) {
+  constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;   // low bytes 00 00 80 C0 | 00 40 80 C0
+  constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;   // high bytes 00 3F 3F 3F | 40 40 40 40
+  const uint32_t m = c & 0x77777777u;
+  const uint32_t mh = m >> 16;
+  const uint32_t lo_a = __byte_perm(kLo0, kLo1, m), hi_a = __byte_perm(kHi0, kHi1, m);
+  const uint32_t lo_b = __byte_perm(kLo0, kLo1, mh), hi_b = __byte_perm(kHi0, kHi1, mh);
+  const uint32_t c4 = c << 4;
+  w[0] = __byte_perm(lo_a, hi_a, 0x5140) | (__byte_perm(c4, c, 0x4000) & 0x80008000u);
+  w[1] = __byte_perm(lo_a, hi_a, 0x7362) | (__byte_perm(c4, c, 0x5010) & 0x80008000u);
+  w[2] = __byte_perm(lo_b, hi_b, 0x5140) | (__byte_perm(c4, c, 0x6020) & 0x80008000u);
+  w[3] = __byte_perm(lo_b, hi_b, 0x7362) | (__byte_perm(c4, c, 0x7030) & 0x80008000u);
+}
+
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t saddr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
+  return v;
+}
+
+__global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_constant__ BParams P) {
+  using namespace w4;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + w4::kBarrierOff);
+  uint64_t *empty = full + RS;
+  uint64_t *cfull = empty + RS;
+  uint64_t *cempty = cfull + CS;
+  uint64_t *acc_full = cempty + CS;
+  uint64_t *acc_empty = acc_full + ACC;
+  uint64_t *drain = acc_empty + ACC;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *never = reinterpret_cast<int *>(tmem_slot + 2);
+
+  const Bf16GemmArgs &a = P.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < CS; ++s) {
+      mbar_init(&cfull[s], kConvWarps);
+      mbar_init(&cempty[s], 1);
+    }
+    for (int s = 0; s < ACC; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensor_map(&P.tmap_a);
+    prefetch_tensor_map(&P.tmap_b);
+    prefetch_tensor_map(&P.tmap_out);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_tiles = (int)(a.N / BN);
+  int64_t rows_used = __ldg(a.padded_offsets + a.E);
+  if (rows_used > a.rows_cap) rows_used = a.rows_cap;
+  if (rows_used < 0) rows_used = 0;
+  const int64_t total = (rows_used / BM) * n_tiles;
+  const int ksteps = (int)(a.K / BK);
+  const int64_t k_atoms = a.K >> 6;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      uint32_t p = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = tile_of(a, t, n_tiles, 0);
+        const int64_t wrow = (int64_t)tl.e * a.N + tl.n0;
+        const uint8_t *sf0 = a.b_sf + (wrow >> 7) * k_atoms * 512;
+        uint32_t st = p % RS, ph = (p / RS) & 1u;
+        for (int kt = 0; kt < ksteps; ++kt, ++p) {
+          if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, a.err, 530)) { ok = false; break; }
+          uint8_t *raw = smem + (size_t)st * kRawBytes;
+          mbar_arrive_expect_tx(&full[st], kRawBytes);
+          tma_load_2d(raw, &P.tmap_a, kt * BK, (int32_t)tl.m0, &full[st]);
+          tma_load_2d(raw + kABytes, &P.tmap_b, kt * (BK / 2), (int32_t)wrow, &full[st]);
+          bulk_load(raw + kABytes + kCodesBytes, sf0 + (int64_t)kt * 512, 512, &full[st]);
+          bulk_load(raw + kABytes + kCodesBytes + 512, sf0 + (k_atoms + kt) * 512, 512, &full[st]);
+          if (++st == RS) { st = 0; ph ^= 1u; }
+        }
+      }
+      for (uint32_t q = p > RS ? p - RS : 0; q < p; ++q)
+        mbar_wait_bounded(&full[q % RS], (q / RS) & 1u, never, a.err, 531);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      const uint64_t dk = smem_desc(0, 16, 1024, 2);
+      const uint32_t idesc = idesc_bf16(0, 0);
+      const uint32_t smem0 = smem_u32(smem);
+      uint32_t p = 0, it = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const uint32_t as = it % ACC;
+        const uint32_t acc = tmem + as * BN;
+        if (!mbar_wait_bounded(&acc_empty[as], ((it / ACC) & 1u) ^ 1u, abort_flag, a.err, 540)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < ksteps; ++kt, ++p) {
+          const uint32_t st = p % RS, cs = p % CS;
+          if (!mbar_wait_bounded(&full[st], (p / RS) & 1u, abort_flag, a.err, 541) ||
+              !mbar_wait_bounded(&cfull[cs], (p / CS) & 1u, abort_flag, a.err, 542)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a16 = (smem0 + st * (uint32_t)kRawBytes) >> 4;
+          const uint64_t b16 = (smem0 + (uint32_t)kConvOff + cs * (uint32_t)kBBytes) >> 4;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(acc, dk | (a16 + kk * 2), dk | (b16 + kk * 2), idesc, (kt | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty[st]);
+          tc_commit(&cempty[cs]);
+        }
+        if (ok) tc_commit(&acc_full[as]);
+      }
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0, never, a.err, 543);
+    }
+  } else if (warp >= kConvWarp0) {
+    // ------------------------------------------------------- converters
+    // Lane l of converter warp w covers K-half (l & 1) of B rows
+    // 32w + l/2 and 32w + 16 + l/2: its 16-byte code loads are contiguous
+    // across the warp, and its 16-byte stores land in distinct banks within
+    // every quarter warp under the 128-byte swizzle.
+    const int cw = warp - kConvWarp0;
+    const int hk = lane & 1;
+    const uint32_t smem0 = smem_u32(smem);
+    int r[2];
+    uint32_t code_off[2], sf_off[2], dst_off[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      r[j] = 32 * cw + 16 * j + (lane >> 1);
+      code_off[j] = (uint32_t)(kABytes + r[j] * 32 + hk * 16);
+      sf_off[j] = (uint32_t)(kABytes + kCodesBytes + (r[j] >> 7) * 512 + (r[j] & 31) * 16 + ((r[j] & 127) >> 5) * 4 +
+                             2 * hk);
+      dst_off[j] = (uint32_t)(r[j] * 128);
+    }
+    uint32_t p = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int kt = 0; kt < ksteps; ++kt, ++p) {
+        const uint32_t st = p % RS, cs = p % CS;
+        if (!mbar_wait_bounded(&full[st], (p / RS) & 1u, abort_flag, a.err, 550) ||
+            !mbar_wait_bounded(&cempty[cs], ((p / CS) & 1u) ^ 1u, abort_flag, a.err, 551)) {
+          ok = false;
+          break;
+        }
+        const uint32_t raw = smem0 + st * (uint32_t)kRawBytes;
+        const uint32_t dst = smem0 + (uint32_t)kConvOff + cs * (uint32_t)kBBytes;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint4 q = ld_shared_v4(raw + code_off[j]);
+          const uint32_t sc = ld_shared_u16(raw + sf_off[j]);
+          const float s0 = ue4m3_value(sc & 0xFFu), s1 = ue4m3_value(sc >> 8);
+          const uint32_t s2[2] = {pack_bf16x2(s0, s0), pack_bf16x2(s1, s1)};
+          const uint32_t cw4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+            e2m1x8_to_bf16x2(cw4[i], w);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w[u] = mul_bf16x2(w[u], s2[i >> 1]);
+            const uint32_t chunk = (uint32_t)(4 * hk + i) ^ (uint32_t)(r[j] & 7);
+            st_shared_v4(dst + dst_off[j] + (chunk << 4), w[0], w[1], w[2], w[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cfull[cs]);
+      }
+    }
+  } else if (warp >= w4::kEpiWarp0) {
+    // -------------------------------------------------------- epilogue
+    const int ew = warp - w4::kEpiWarp0;
+    const int quad = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
+    uint8_t *stg = smem + w4::kStagingOff + (size_t)ew * kStagingPerWarp;
+    const uint32_t stg_addr = smem_u32(stg);
+    uint32_t chunk_id = 0, it = 0;
+    auto store_box = [&](const uint32_t (&w16)[16], int32_t x, int32_t y) {
+      const uint32_t box = stg_addr + (chunk_id & 1u) * 2048;
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      stage_row(box, lane, w16);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&P.tmap_out, stg + (chunk_id & 1u) * 2048, x, y);
+        bulk_commit_group();
+      }
+      ++chunk_id;
+    };
+    const int64_t rows_total = (int64_t)__ldg(a.offsets + a.E);
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const Tile tl = tile_of(a, t, n_tiles, 0);
+      const uint32_t as = it % ACC;
+      const float scale = __ldg(a.s_dec_w + tl.e);
+      if (!mbar_wait_bounded(&acc_full[as], (it / ACC) & 1u, abort_flag, a.err, 560)) break;
+      tc_fence_after();
+      const uint32_t tacc = tlane + as * BN;
+      if (a.epilogue == kBfSwiGLUFwd) {
+        // gate columns [half*64, +64), up columns [128 + half*64, +64) of the
+        // tile (the gate_up weight rows are interleaved in blocks of 128);
+        // h columns n0/2 + half*64 + [0, 64), every padded row of the slab
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t vg[32], vu[32];
+          tmem_ld_32cols(tacc + half * 64 + c * 32, vg);
+          tmem_ld_32cols(tacc + 128 + half * 64 + c * 32, vu);
+          tmem_ld_wait();
+          if (c == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[as]);
+          }
+          uint32_t w16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float hh[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float g = __fmul_rn(__uint_as_float(vg[2 * i + q]), scale);
+              const float u = __fmul_rn(__uint_as_float(vu[2 * i + q]), scale);
+              // silu(g) = g / (1 + e^-g) with the fast exponential and
+              // division (~2^-21 relative, far below a BF16 ulp of h)
+              hh[q] = __fmul_rn(__fdividef(g, 1.0f + __expf(-g)), u);
+            }
+            w16[i] = pack_bf16x2(hh[0], hh[1]);
+          }
+          store_box(w16, (int32_t)(tl.n0 / 2 + half * 64 + c * 32), (int32_t)(tl.m0 + quad * 32));
+        }
+      } else {
+        const int64_t g_pad = __ldg(a.padded_offsets + tl.e);
+        const int64_t g_off = __ldg(a.offsets + tl.e);
+        const int64_t g_cnt = (int64_t)__ldg(a.offsets + tl.e + 1) - g_off;
+        const int64_t rel = tl.m0 - g_pad + quad * 32 + lane;
+        const bool valid = rel < g_cnt && g_off + rel < rows_total;
+        const int64_t prow = tl.m0 + quad * 32 + lane;
+        const int64_t orow = a.out_padded ? prow : g_off + rel;
+        const bool slab_full = a.out_padded || (tl.m0 - g_pad) + quad * 32 + 32 <= g_cnt;
+        const int64_t slab_row = a.out_padded ? tl.m0 + quad * 32 : g_off + (tl.m0 - g_pad) + quad * 32;
+        const int64_t col0 = tl.n0 + half * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld_32cols(tacc + half * 128 + c * 32, v);
+          tmem_ld_wait();
+          if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[as]);
+          }
+          uint32_t w16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w16[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * i]), scale),
+                                 __fmul_rn(__uint_as_float(v[2 * i + 1]), scale));
+          if (slab_full) {
+            store_box(w16, (int32_t)(col0 + c * 32), (int32_t)slab_row);
+          } else if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_bf16) + orow * a.N + col0 +
+                                                   c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+          }
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
+
+static cudaError_t launch_w4a16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
+  if (a.mode != kBfRows || a.b_mn || a.s_dec_w == nullptr || a.out_bf16 == nullptr || a.K % BK != 0 ||
+      (a.epilogue != kBfStore && a.epilogue != kBfSwiGLUFwd) || (a.epilogue == kBfSwiGLUFwd && !a.out_padded))
+    return cudaErrorInvalidValue;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(k_w4a16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)w4::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
+  }
+  BParams P;
+  P.a = a;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.K, (uint64_t)a.rows_cap, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!encode_2d_map(&P.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b, (uint64_t)(a.K / 2), (uint64_t)(a.E * a.N),
+                     BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const uint64_t out_cols = a.epilogue == kBfSwiGLUFwd ? (uint64_t)(a.N / 2) : (uint64_t)a.N;
+  if (!encode_2d_map(&P.tmap_out, BF, 2, a.out_bf16, out_cols, (uint64_t)a.rows_cap, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  const int64_t tiles = (a.rows_cap / BM) * (a.N / BN);
+  int64_t grid = num_sms();
+  if (grid > tiles) grid = tiles;
+  if (grid < 1) grid = 1;
+  k_w4a16_gemm<<<(unsigned)grid, w4::kThreads, w4::kSmemBytes, s>>>(P);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
   if (a.rows_cap <= 0 || a.N % BN != 0) return a.rows_cap <= 0 ? cudaSuccess : cudaErrorInvalidValue;
+  if (a.b_sf != nullptr) return launch_w4a16_gemm(a, s);
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);

@@ -136,6 +136,7 @@ enum Bf16GemmMode : int {
 enum Bf16Epilogue : int {
   kBfStore = 0,       // BF16 and/or FP32 output
   kBfSwiGLUBwd = 1,   // backward of SwiGLU and of the combine's dot (see gemm_bf16.cu)
+  kBfSwiGLUFwd = 2,   // W4A16 gate_up: h = BF16(silu(g) u) of the scaled accumulator
 };
 
 struct Bf16GemmArgs {
@@ -159,12 +160,18 @@ struct Bf16GemmArgs {
   void *d_gu = nullptr;         // BF16 [rows_cap][2I] (out)
   void *hw = nullptr;           // BF16 [rows_cap][I] (out): w * BF16(silu(g) u)
   float *dw_part = nullptr;     // [rows_cap][I/128] (out): partial <dh', h> per 128 columns
+  // W4A16 (kBfRows, B K-major): B is NVFP4 -- b holds the E2M1 codes
+  // [E][N][K/2], b_sf the UE4M3 block scales in the MMA atom layout, s_dec_w
+  // the per-expert decode scale applied to the accumulator in the epilogue
+  const uint8_t *b_sf = nullptr;
+  const float *s_dec_w = nullptr;
   int *err = nullptr;
 };
 cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s);
 
 // Backward helpers: gather x and dy rows into the padded grouped layout
-// (zeros on padding rows), the row weights, and ones for the dx combine.
+// (zeros on padding rows), the row weights, and ones for the dx combine
+// (dy / dy_rows, w_rows and ones may be null).
 struct BwdGatherParams {
   const void *x, *dy;
   const float *topk_w;

@@ -77,6 +77,11 @@ _SIGS = {
                                                            ctypes.POINTER(_i64)]),
     "moe_expert_layer_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp,
                                          _vp, _vp, _vp, _vp, _u32, _vp, _sz, _vp]),
+    "moe_expert_layer_w4a16_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32, _u32]),
+    "moe_expert_layer_w4a16_workspace_offsets": (_i32, [_i64, _i64, _i64, _i32, _i32, _u32,
+                                                        ctypes.POINTER(_i64)]),
+    "moe_expert_layer_w4a16": (_i32, [_vp, _vp, _vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights),
+                                      _i64, _i64, _i64, _i32, _i32, _vp, _u32, _vp, _sz, _vp]),
     "nvfp4moe_num_sms": (_i32, []),
 }
 
@@ -391,6 +396,62 @@ def backward_views(workspace: torch.Tensor, T, H, I, E, k, flags=0) -> dict:
     if flags & BWD_KEEP_DH:
         v["dh"] = view("dh", cap * I * 4, torch.float32, (cap, I))
     return v
+
+
+# ---------------------------------------------------------------- W4A16 --
+
+def moe_expert_layer_w4a16_workspace_size(T, H, I, E, k, flags=0) -> int:
+    return int(lib().moe_expert_layer_w4a16_workspace_size(T, H, I, E, k, flags))
+
+
+_W4A16_REGIONS = ["err", "offsets", "padded_offsets", "perm", "inv_perm", "x_rows", "h", "d"]
+
+
+def moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k, flags=0) -> dict:
+    arr = (ctypes.c_int64 * 16)()
+    _check(lib().moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k, flags, arr),
+           "moe_expert_layer_w4a16_workspace_offsets")
+    out = {name: int(arr[i]) for i, name in enumerate(_W4A16_REGIONS)}
+    out["rows_cap"] = int(arr[14])
+    out["total"] = int(arr[15])
+    return out
+
+
+def moe_expert_layer_w4a16(x, topk_idx, topk_w, w_gate_up: NVFP4Weights, w_down: NVFP4Weights, y,
+                           workspace, flags=0, stream=None):
+    """moe_expert_layer_w4a16: BF16 activations, the same prepared NVFP4
+    weights as moe_expert_layer."""
+    _dev(x, topk_idx, topk_w, y, workspace)
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    I = w_down.K
+    gu, dn = w_gate_up.struct(), w_down.struct()
+    _check(lib().moe_expert_layer_w4a16(_p(x), _p(topk_idx), _p(topk_w), ctypes.byref(gu), ctypes.byref(dn),
+                                        T, H, I, w_down.E, k, _p(y), flags, _p(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "moe_expert_layer_w4a16")
+
+
+def w4a16_views(workspace: torch.Tensor, T, H, I, E, k) -> dict:
+    """Typed views of the W4A16 workspace's regions (for inspection in tests)."""
+    o = moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k)
+    cap = o["rows_cap"]
+    R = T * k
+    ws = workspace
+
+    def view(name, nbytes, dtype, shape):
+        return ws[o[name]:o[name] + nbytes].view(dtype).view(*shape)
+
+    return {
+        "rows_cap": cap,
+        "offsets": view("offsets", (E + 1) * 4, torch.int32, (E + 1,)),
+        "padded_offsets": view("padded_offsets", (E + 1) * 4, torch.int32, (E + 1,)),
+        "perm": view("perm", R * 4, torch.int32, (R,)),
+        "inv_perm": view("inv_perm", R * 4, torch.int32, (T, k)),
+        "x_rows": view("x_rows", cap * H * 2, torch.bfloat16, (cap, H)),
+        "h": view("h", cap * I * 2, torch.bfloat16, (cap, I)),
+        "d": view("d", R * H * 2, torch.bfloat16, (R, H)),
+    }
 
 
 def nvfp4moe_encode_e2m1(y: torch.Tensor, codes: torch.Tensor, stream=None):
