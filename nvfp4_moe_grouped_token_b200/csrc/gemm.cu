@@ -115,6 +115,7 @@ struct Cfg {
                                      ((uint32_t)(BM >> 4) << 24);
   static_assert(ACC * BN + STAGES * (16 + 16 * kNAtoms) <= (int)kTmemCols, "TMEM budget");
   static_assert(kSmemMax <= 232448, "shared memory budget");
+  static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 12 <= 192, "pipeline barriers overrun their area");
 };
 
 using CfgGateUp = Cfg<256, 3, 1>;
@@ -374,8 +375,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *never = reinterpret_cast<int *>(tmem_slot + 2);   // an abort flag nothing raises
-  uint64_t *req_bar = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 128);   // [2 workers][2]
-  uint32_t *mt_done = reinterpret_cast<uint32_t *>(smem + C::kBarrierOff + 320);
+  // barrier area: pipeline barriers and flags [0, 192), the fused
+  // requantization's worker barriers [192, 224), its epilogue-warp barriers
+  // [224, 352), its counters at 384
+  uint64_t *req_bar = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 192);   // [2 workers][2]
+  uint32_t *mt_done = reinterpret_cast<uint32_t *>(smem + C::kBarrierOff + 384);
   uint32_t *slab_next = mt_done + 1;
   int32_t *s_pad = reinterpret_cast<int32_t *>(smem + C::kOffsetsOff);
   int32_t *s_off = s_pad + (P.a.E + 1);
@@ -787,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       ReqStage rs;
       rs.buf[0] = stg;
       rs.buf[1] = stg + kStagingPerWarp / 2;
-      rs.bar[0] = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 160) + 2 * ew;
+      rs.bar[0] = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 224) + 2 * ew;
       rs.bar[1] = rs.bar[0] + 1;
       rs.piece = kStagingPerWarp / 2;
       rs.loads[0] = rs.loads[1] = 0;
@@ -900,7 +904,10 @@ cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
   if (a.rows_cap <= 0) return cudaSuccess;
   // both GEMMs use 128 x 256 tiles with one accumulator (the SwiGLU epilogue
-  // reads gate and up from the two 128-column halves of a tile)
+  // reads gate and up from the two 128-column halves of a tile).  128 x 128
+  // tiles with two accumulators (Cfg<128, 4, 2>) also pass the parity tests
+  // but run the down GEMM of the Qwen3-30B-A3B-shaped layer in 239 us
+  // instead of 183 us: its cost is per K-step, not the accumulator hand-over.
   if (a.epilogue == kEpiSwiGLU) return launch_cfg<CfgGateUp>(a, s);
   return launch_cfg<CfgDown>(a, s);
 }

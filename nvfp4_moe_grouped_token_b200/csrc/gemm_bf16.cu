@@ -455,6 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
 // (at most 2 + 4 significant bits, exponents well inside the range), so the
 // converted operand is exactly the dequantized weight divided by the
 // per-expert S_dec, which the epilogue applies to the FP32 accumulator.
+// (The decode multiplies code * 2^120 by scale * 2^-120 in BF16; the second
+// factor is a BF16 subnormal for subnormal UE4M3 scales, which the BF16
+// multiply keeps.)
 //
 //   raw ring (4 stages): A 16 KB (TMA, swizzled) + codes 8 KB (TMA, 256 rows
 //     x 32 bytes, unswizzled) + scales 1 KB (two 512-byte atoms, bulk copies)
@@ -479,23 +482,43 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kConvWarps * 32 * 2 == 2 * BN, "each converter lane covers two half rows");
 }  // namespace w4
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 // Eight E2M1 codes (one word; element 2b is the low nibble of byte b) ->
-// four BF16 pairs in element order.  The 3-bit magnitude indexes two
-// eight-entry byte tables held in registers (the high and the low byte of the
-// BF16 value of 0, 0.5, 1, 1.5, 2, 3, 4, 6); the code's sign bit becomes
-// bit 15 or 31 of its pair.
+// four BF16 pairs in element order holding code * 2^120.  The 3-bit
+// magnitude indexes two eight-entry byte tables held in registers: the low
+// and the high byte of the BF16 value of 2^120 * {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+// Each code's sign bit is moved to bit 7 of its high byte on the way (one
+// byte permute gathers the four sign bits of four codes).
 __device__ __forceinline__ void e2m1x8_to_bf16x2(uint32_t c, uint32_t (&w)[4]) {
   constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;   // low bytes 00 00 80 C0 | 00 40 80 C0
-  constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;   // high bytes 00 3F 3F 3F | 40 40 40 40
+  constexpr uint32_t kHi0 = 0x7B7B7B00u, kHi1 = 0x7C7C7C7Cu;   // high bytes 00 7B 7B 7B | 7C 7C 7C 7C
   const uint32_t m = c & 0x77777777u;
   const uint32_t mh = m >> 16;
-  const uint32_t lo_a = __byte_perm(kLo0, kLo1, m), hi_a = __byte_perm(kHi0, kHi1, m);
-  const uint32_t lo_b = __byte_perm(kLo0, kLo1, mh), hi_b = __byte_perm(kHi0, kHi1, mh);
   const uint32_t c4 = c << 4;
-  w[0] = __byte_perm(lo_a, hi_a, 0x5140) | (__byte_perm(c4, c, 0x4000) & 0x80008000u);
-  w[1] = __byte_perm(lo_a, hi_a, 0x7362) | (__byte_perm(c4, c, 0x5010) & 0x80008000u);
-  w[2] = __byte_perm(lo_b, hi_b, 0x5140) | (__byte_perm(c4, c, 0x6020) & 0x80008000u);
-  w[3] = __byte_perm(lo_b, hi_b, 0x7362) | (__byte_perm(c4, c, 0x7030) & 0x80008000u);
+  const uint32_t lo_a = prmt(kLo0, kLo1, m), lo_b = prmt(kLo0, kLo1, mh);
+  // byte j of the sign word holds code j's sign at bit 7: bytes c4.b0, c.b0, c4.b1, c.b1 (codes 0-3)
+  const uint32_t hi_a = prmt(kHi0, kHi1, m) | (prmt(c4, c, 0x5140) & 0x80808080u);
+  const uint32_t hi_b = prmt(kHi0, kHi1, mh) | (prmt(c4, c, 0x7362) & 0x80808080u);
+  w[0] = prmt(lo_a, hi_a, 0x5140);
+  w[1] = prmt(lo_a, hi_a, 0x7362);
+  w[2] = prmt(lo_b, hi_b, 0x5140);
+  w[3] = prmt(lo_b, hi_b, 0x7362);
+}
+
+// Two UE4M3 block scales (bytes of sc) -> BF16 pairs (s0, s0) and (s1, s1)
+// holding scale * 2^-120: a UE4M3 code b shifted left by 4 is, read as BF16
+// bits, exactly its value times 2^-120 (normal codes: exponent e - 7 + 127 -
+// 120; subnormal codes m * 2^-9 become BF16 subnormals m * 2^-129).  Times
+// the table's 2^120 the products are exactly code * scale.
+__device__ __forceinline__ void ue4m3x2_to_bf16x2(uint32_t sc, uint32_t &s0, uint32_t &s1) {
+  const uint32_t u = prmt(sc, 0u, 0x4140) << 4;   // b0 << 4 in the low half, b1 << 4 in the high half
+  s0 = prmt(u, 0u, 0x1010);
+  s1 = prmt(u, 0u, 0x3232);
 }
 
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
@@ -641,15 +664,15 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     const int cw = warp - kConvWarp0;
     const int hk = lane & 1;
     const uint32_t smem0 = smem_u32(smem);
-    int r[2];
-    uint32_t code_off[2], sf_off[2], dst_off[2];
+    uint32_t code_off[2], sf_off[2], dst_off[2][4];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      r[j] = 32 * cw + 16 * j + (lane >> 1);
-      code_off[j] = (uint32_t)(kABytes + r[j] * 32 + hk * 16);
-      sf_off[j] = (uint32_t)(kABytes + kCodesBytes + (r[j] >> 7) * 512 + (r[j] & 31) * 16 + ((r[j] & 127) >> 5) * 4 +
-                             2 * hk);
-      dst_off[j] = (uint32_t)(r[j] * 128);
+      const int r = 32 * cw + 16 * j + (lane >> 1);
+      code_off[j] = (uint32_t)(kABytes + r * 32 + hk * 16);
+      sf_off[j] = (uint32_t)(kABytes + kCodesBytes + (r >> 7) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + 2 * hk);
+      // 16-byte chunk 4hk + i of row r under the 128-byte swizzle
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst_off[j][i] = (uint32_t)(r * 128) + ((uint32_t)((4 * hk + i) ^ (r & 7)) << 4);
     }
     uint32_t p = 0;
     bool ok = true;
@@ -663,21 +686,25 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
         }
         const uint32_t raw = smem0 + st * (uint32_t)kRawBytes;
         const uint32_t dst = smem0 + (uint32_t)kConvOff + cs * (uint32_t)kBBytes;
+        uint4 q[2];
+        uint32_t sc[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const uint4 q = ld_shared_v4(raw + code_off[j]);
-          const uint32_t sc = ld_shared_u16(raw + sf_off[j]);
-          const float s0 = ue4m3_value(sc & 0xFFu), s1 = ue4m3_value(sc >> 8);
-          const uint32_t s2[2] = {pack_bf16x2(s0, s0), pack_bf16x2(s1, s1)};
-          const uint32_t cw4[4] = {q.x, q.y, q.z, q.w};
+          q[j] = ld_shared_v4(raw + code_off[j]);
+          sc[j] = ld_shared_u16(raw + sf_off[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          uint32_t s2[2];
+          ue4m3x2_to_bf16x2(sc[j], s2[0], s2[1]);
+          const uint32_t cw4[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t w[4];
             e2m1x8_to_bf16x2(cw4[i], w);
 #pragma unroll
             for (int u = 0; u < 4; ++u) w[u] = mul_bf16x2(w[u], s2[i >> 1]);
-            const uint32_t chunk = (uint32_t)(4 * hk + i) ^ (uint32_t)(r[j] & 7);
-            st_shared_v4(dst + dst_off[j] + (chunk << 4), w[0], w[1], w[2], w[3]);
+            st_shared_v4(dst + dst_off[j][i], w[0], w[1], w[2], w[3]);
           }
         }
         fence_proxy_async_smem();

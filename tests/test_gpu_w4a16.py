@@ -155,3 +155,23 @@ def test_w4a16_is_deterministic():
     L.ws.zero_()
     L.run()
     assert torch.equal(L.y.view(torch.int16), y0.view(torch.int16))
+
+
+def test_w4a16_subnormal_block_scales():
+    """One weight of 2000 per matrix beside N(0, 0.02) weights: most blocks'
+    UE4M3 scales are subnormal (m * 2^-9).  The converter decodes a scale as
+    BF16 bits (a BF16 subnormal for these) and multiplies it in BF16; the
+    products must still be exactly code * scale."""
+    cfg = workloads.LayerConfig("subnormal_w4a16", T=200, H=256, I=256, E=2, k=1, seed=33)
+    inp = workloads.layer_inputs(cfg)
+    for key in ("w_gate_up", "w_down"):
+        w = inp[key].clone()
+        w[:, 0, 0] = 2000.0
+        inp[key] = w
+    L = W4(cfg, inp)
+    for prep in (L.wgu, L.wdn):
+        sf = prep.sf.cpu().numpy()
+        sub = (((sf >> 3) & 0xF) == 0) & ((sf & 7) != 0)
+        assert sub.mean() > 0.5, sub.mean()
+    L.run()
+    L.check()
