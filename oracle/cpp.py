@@ -62,6 +62,10 @@ _SIGS = {
     "orc_swiglu_backward": (None, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "orc_expert_layer_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _vp, _vp,
                                          _vp, _vp]),
+    "orc_mxfp8_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp]),
+    "orc_mxfp8_dequantize": (None, [_vp, _vp, _i64, _i64, _vp]),
+    "orc_expert_layer_w4a8": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
+                                     ctypes.POINTER(_LayerOut)]),
     "orc_expert_layer_w4a16": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
                                       ctypes.POINTER(_LayerOut)]),
     "orc_expert_layer": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32,
@@ -321,10 +325,41 @@ def expert_layer_backward(x, topk_idx, topk_w, w_gate_up, w_down, dy) -> dict:
     return out
 
 
+def mxfp8_quantize(x):
+    """R17: MXFP8 codes (E4M3, bit 7 the sign) [M][K] and E8M0 scales [M][K/32]."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    codes = np.empty((M, K), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    if lib().orc_mxfp8_quantize(_p(x), M, K, _p(codes), _p(scales)) != 0:
+        raise ValueError("K must be a multiple of 32")
+    return codes, scales
+
+
+def mxfp8_dequantize(codes, scales) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    M, K = codes.shape
+    out = np.empty((M, K), np.float64)
+    lib().orc_mxfp8_dequantize(_p(codes), _p(scales), M, K, _p(out))
+    return out
+
+
+def expert_layer_w4a8(x, topk_idx, topk_w, w_gate_up, w_down) -> dict:
+    """R20: the layer with NVFP4 weights and MXFP8 activations (x and h).
+    Returns y, offsets, perm, inv_perm, h (BF16 before its MXFP8
+    requantization, sorted rows) and d."""
+    return _layer_variant("orc_expert_layer_w4a8", x, topk_idx, topk_w, w_gate_up, w_down)
+
+
 def expert_layer_w4a16(x, topk_idx, topk_w, w_gate_up, w_down) -> dict:
     """R19: the layer with BF16 activations and NVFP4 weights (x not
     quantized, h not requantized).  Returns y, offsets, perm, inv_perm, h
     (BF16, sorted rows) and d."""
+    return _layer_variant("orc_expert_layer_w4a16", x, topk_idx, topk_w, w_gate_up, w_down)
+
+
+def _layer_variant(fn, x, topk_idx, topk_w, w_gate_up, w_down) -> dict:
     x = _c(x, np.float32)
     idx = _c(topk_idx, np.int32)
     tw = _c(topk_w, np.float32)
@@ -340,8 +375,7 @@ def expert_layer_w4a16(x, topk_idx, topk_w, w_gate_up, w_down) -> dict:
          "inv_perm": np.empty((T, k), np.int32), "h": np.empty((R, I), np.float32), "d": np.empty((R, H), np.float32)}
     fields = {name: arr.ctypes.data for name, arr in o.items()}
     st = _LayerOut(**fields)
-    rc = lib().orc_expert_layer_w4a16(_p(x), _p(idx), _p(tw), _p(wgu), _p(wdn), T, H, I, E, k, threads(),
-                                      ctypes.byref(st))
+    rc = getattr(lib(), fn)(_p(x), _p(idx), _p(tw), _p(wgu), _p(wdn), T, H, I, E, k, threads(), ctypes.byref(st))
     if rc != 0:
-        raise ValueError("orc_expert_layer_w4a16: bad shape or routing entry")
+        raise ValueError(f"{fn}: bad shape or routing entry")
     return o

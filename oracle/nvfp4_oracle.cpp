@@ -47,6 +47,16 @@
 //       the same NVFP4 weights, BF16 activations: x is not quantized and h is
 //       not requantized; G = x W_gu^T on the dequantized weights in fp64,
 //       h = BF16(silu(g) u), D = BF16(h W_dn^T), then the same combine.
+//   R17 MXFP8 (W4A8 activations; the pages name the format only, this is the
+//       public OCP MX definition): blocks of 32 consecutive elements along a
+//       row share an E8M0 scale 2^s, s = floor(log2(block amax)) - 8
+//       clamped to [-127, 127] (-127 for an all-zero block); elements are
+//       E4M3(v / 2^s), round to nearest even, saturating at +-448, sign kept
+//       (a negative value that rounds to 0 is code 0x80).
+//   R20 W4A8 variant (the same paragraph 3 of the aib.vote report): the W4A4
+//       layer's NVFP4 weights, activations x and h in MXFP8 (R17), each
+//       dequantized exactly; h = BF16(silu(g) u) is the requantization input
+//       as in R11.  Everything else as R19.
 //   R16 backward, BF16-backward mode (www.aib.vote "miniTE report, NVFP4 RL
 //       stability", paragraph 1 times "NVFP4 forward, BF16 backward" without
 //       formulas): the exact gradient of the unquantized layer on its BF16
@@ -513,6 +523,97 @@ int orc_expert_layer_w4a16(const float *x, const int32_t *topk_idx, const float 
   orc_round_bf16_n(hd.data(), R * I, h.data());
   for (int64_t i = 0; i < R * I; ++i) hb[i] = h[i];
   orc_grouped_gemm(hb.data(), off.data(), E, wdn.data(), H, I, dd.data(), nullptr, threads);
+  std::vector<float> d(R * H);
+  orc_round_bf16_n(dd.data(), R * H, d.data());
+  orc_combine(d.data(), H, inv.data(), topk_w, T, k, out->y);
+  auto put = [](auto *dst, const auto &src) {
+    if (dst != nullptr) std::copy(src.begin(), src.end(), dst);
+  };
+  put(out->offsets, off);
+  put(out->padded_offsets, pad);
+  put(out->perm, perm);
+  put(out->inv_perm, inv);
+  put(out->h, h);
+  put(out->d, d);
+  return 0;
+}
+
+// R17: MXFP8 quantization of rows x [M][K] (K % 32 == 0): codes [M][K]
+// (E4M3, bit 7 the sign) and scales [M][K/32] (E8M0 code = s + 127).
+int orc_mxfp8_quantize(const float *x, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales) {
+  if (K % 32 != 0) return -1;
+  for (int64_t r = 0; r < M; ++r) {
+    for (int64_t b = 0; b < K / 32; ++b) {
+      const float *v = x + r * K + b * 32;
+      double amax = 0.0;
+      for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs((double)v[i]));
+      int s = -127;
+      if (amax > 0.0) {
+        int e2;
+        std::frexp(amax, &e2);        // amax = f * 2^e2, f in [0.5, 1): floor(log2 amax) = e2 - 1
+        s = std::min(127, std::max(-127, (e2 - 1) - 8));
+      }
+      scales[r * (K / 32) + b] = (uint8_t)(s + 127);
+      for (int i = 0; i < 32; ++i) {
+        const double y = std::ldexp((double)v[i], -s);   // exact: a power-of-two scale
+        const int mag = nearest_even(std::fabs(y), kUE4M3.v, 127);
+        codes[r * K + b * 32 + i] = (uint8_t)(mag | (std::signbit(y) ? 0x80 : 0));
+      }
+    }
+  }
+  return 0;
+}
+
+void orc_mxfp8_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t M, int64_t K, double *out) {
+  for (int64_t r = 0; r < M; ++r)
+    for (int64_t c = 0; c < K; ++c) {
+      const uint8_t q = codes[r * K + c];
+      const double m = ue4m3_value(q & 0x7F);
+      out[r * K + c] = std::ldexp((q & 0x80) ? -m : m, (int)scales[r * (K / 32) + c / 32] - 127);
+    }
+}
+
+// R20: the W4A8 variant -- NVFP4 weights, MXFP8 activations (x and h).
+// Outputs y, the permutation, h (BF16 before its MXFP8 requantization,
+// sorted rows) and D.
+int orc_expert_layer_w4a8(const float *x, const int32_t *topk_idx, const float *topk_w, const float *w_gate_up,
+                          const float *w_down, int64_t T, int64_t H, int64_t I, int E, int k, int threads,
+                          OrcLayerOut *out) {
+  if (H % 32 != 0 || I % 32 != 0 || out == nullptr || out->y == nullptr) return -1;
+  const int64_t R = T * k;
+  std::vector<int32_t> off(E + 1), pad(E + 1), perm(R), inv(R);
+  if (orc_permutation(topk_idx, T, k, E, off.data(), pad.data(), perm.data(), inv.data()) != 0) return -1;
+  // x: MXFP8 per token, dequantized exactly
+  std::vector<uint8_t> xc(T * H), xs(T * (H / 32));
+  orc_mxfp8_quantize(x, T, H, xc.data(), xs.data());
+  std::vector<double> xd(T * H);
+  orc_mxfp8_dequantize(xc.data(), xs.data(), T, H, xd.data());
+  std::vector<double> a(R * H);
+  for (int64_t p = 0; p < R; ++p) {
+    const int64_t t = perm[p] / k;
+    for (int64_t c = 0; c < H; ++c) a[p * H + c] = xd[t * H + c];
+  }
+  std::vector<double> wgu((int64_t)E * 2 * I * H), wdn((int64_t)E * H * I);
+  for (int e = 0; e < E; ++e) {
+    std::vector<uint8_t> q(2 * I * H / 2), sc(2 * I * H / 16);
+    float sd, am;
+    orc_quantize(w_gate_up + (int64_t)e * 2 * I * H, 2 * I, H, 0, nullptr, q.data(), sc.data(), &sd, &am);
+    orc_dequantize(q.data(), sc.data(), &sd, 2 * I, H, 0, &wgu[(int64_t)e * 2 * I * H]);
+    std::vector<uint8_t> q2(H * I / 2), s2(H * I / 16);
+    orc_quantize(w_down + (int64_t)e * H * I, H, I, 0, nullptr, q2.data(), s2.data(), &sd, &am);
+    orc_dequantize(q2.data(), s2.data(), &sd, H, I, 0, &wdn[(int64_t)e * H * I]);
+  }
+  std::vector<double> gu(R * 2 * I), hd(R * I), dd(R * H);
+  orc_grouped_gemm(a.data(), off.data(), E, wgu.data(), 2 * I, H, gu.data(), nullptr, threads);
+  orc_swiglu(gu.data(), R, I, hd.data());
+  std::vector<float> h(R * I);
+  orc_round_bf16_n(hd.data(), R * I, h.data());
+  // h: MXFP8 per row, dequantized exactly
+  std::vector<uint8_t> hc(R * I), hs(R * (I / 32));
+  orc_mxfp8_quantize(h.data(), R, I, hc.data(), hs.data());
+  std::vector<double> hq(R * I);
+  orc_mxfp8_dequantize(hc.data(), hs.data(), R, I, hq.data());
+  orc_grouped_gemm(hq.data(), off.data(), E, wdn.data(), H, I, dd.data(), nullptr, threads);
   std::vector<float> d(R * H);
   orc_round_bf16_n(dd.data(), R * H, d.data());
   orc_combine(d.data(), H, inv.data(), topk_w, T, k, out->y);

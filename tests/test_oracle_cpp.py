@@ -368,3 +368,78 @@ def test_w4a16_layer_against_per_token_brute_force():
             acc = acc + float(tw[t, j]) * d.astype(np.float64)
         y[t] = nvfp4.round_to_bf16(acc)
     assert np.array_equal(out["y"], y)
+
+
+def test_mxfp8_hand_derived_codes():
+    """R17 on hand-derived values.  Block amax 1.9: s = floor(log2 1.9) - 8 =
+    -8 (E8M0 code 119), so elements are scaled by 256:
+      1.9   -> 486.4 > 448: saturates to 448 = E4M3 (e 15, m 6) = 0x7E
+      0.3   -> 76.8: binade [64, 128) in steps of 8, nearest 80 = (e 13, m 2) = 0x6A
+      -0.001 -> -0.256: binade [0.25, 0.5) in steps of 1/32, nearest 0.25 = (e 5, m 0), sign -> 0xA8
+      1.0   -> 256 = (e 15, m 0) = 0x78
+      -1e-6 -> -2.56e-4 < half the least subnormal 2^-9: -0 = 0x80
+    An all-zero block takes s = -127 (code 0) and +0 codes."""
+    x = np.zeros((1, 64), np.float32)
+    x[0, :5] = [1.9, 0.3, -0.001, 1.0, -1e-6]
+    codes, scales = cpp.mxfp8_quantize(x)
+    assert list(codes[0, :5]) == [0x7E, 0x6A, 0xA8, 0x78, 0x80]
+    assert not codes[0, 5:32].any() and not codes[0, 32:].any()
+    assert list(scales[0]) == [119, 0]
+    back = cpp.mxfp8_dequantize(codes, scales)
+    assert list(back[0, :5]) == [448 / 256, 80 / 256, -0.25 / 256, 1.0, 0.0]
+    assert math.copysign(1.0, back[0, 4]) == -1.0
+
+
+def test_mxfp8_matches_the_numpy_reading():
+    """The C++ and numpy statements of R17 agree code for code, on normal
+    data, wide dynamic range, BF16 subnormals and all-zero blocks (the numpy
+    one is pinned on its own in test_oracle_mxfp8.py)."""
+    from oracle import mxfp8
+    rng = np.random.default_rng(71)
+    x = rng.standard_normal((64, 256)) * np.exp2(rng.integers(-30, 30, (64, 1)))
+    x[3] = 0.0
+    x[5, :32] = rng.standard_normal(32) * 2.0 ** -130
+    x[7, 7] = 3e38
+    x = nvfp4.round_to_bf16(x).astype(np.float32)
+    c1, s1 = cpp.mxfp8_quantize(x)
+    c2, s2 = mxfp8.quantize(x)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    assert np.array_equal(cpp.mxfp8_dequantize(c1, s1), mxfp8.dequantize(c2, s2))
+
+
+def test_w4a8_layer_against_per_token_brute_force():
+    """R20 (NVFP4 weights, MXFP8 x and h): the grouped path against a
+    per-(token, slot) loop with exactly rounded dot products."""
+    rng = np.random.default_rng(62)
+    T, H, I, E, k = 10, 64, 64, 5, 2
+    x = nvfp4.round_to_bf16(rng.standard_normal((T, H)))
+    idx = np.stack([rng.choice(4, k, replace=False) for _ in range(T)]).astype(np.int32)   # expert 4 empty
+    tw = rng.random((T, k)).astype(np.float32)
+    w_gu = nvfp4.round_to_bf16(rng.standard_normal((E, 2 * I, H)) * 0.05)
+    w_dn = nvfp4.round_to_bf16(rng.standard_normal((E, H, I)) * 0.05)
+    out = cpp.expert_layer_w4a8(x, idx, tw, w_gu, w_dn)
+
+    def wq(w):
+        q = cpp.quantize(w, False)
+        return cpp.dequantize(q["q"], q["sf"], q["s_dec"])
+
+    def qdq(v):
+        return cpp.mxfp8_dequantize(*cpp.mxfp8_quantize(np.asarray(v, np.float32)[None, :]))[0]
+
+    y = np.zeros((T, H), np.float32)
+    for t in range(T):
+        xq = qdq(x[t])
+        acc = np.zeros(H)
+        for j in range(k):
+            e = int(idx[t, j])
+            wgu, wdn = wq(w_gu[e]), wq(w_dn[e])
+            g = np.array([math.fsum(xq * wgu[n]) for n in range(2 * I)])
+            h = nvfp4.round_to_bf16(g[:I] / (1.0 + np.exp(-g[:I])) * g[I:])
+            pos = int(out["inv_perm"][t, j])
+            assert np.array_equal(out["h"][pos], h.astype(np.float32)), (t, j)
+            hq = qdq(h)
+            d = nvfp4.round_to_bf16(np.array([math.fsum(hq * wdn[n]) for n in range(H)]))
+            assert np.array_equal(out["d"][pos], d), (t, j)
+            acc = acc + float(tw[t, j]) * d.astype(np.float64)
+        y[t] = nvfp4.round_to_bf16(acc)
+    assert np.array_equal(out["y"], y)
