@@ -405,6 +405,12 @@ int moe_expert_layer_backward(const void *x, const int32_t *topk_idx,
                               void *workspace, size_t workspace_bytes,
                               nvfp4moe_stream_t stream);
 
+/* The CUDA error code behind the last NVFP4MOE_ERR_CUDA returned on this host
+ * thread (0 if none), with its name, description and the source line of the
+ * failing call written to buf (NUL-terminated, at most len bytes; buf may be
+ * NULL). */
+int nvfp4moe_last_cuda_error(char *buf, size_t len);
+
 /* --------------------------------------------------------------- W4A16 -- */
 /* The MoE expert layer with BF16 activations and NVFP4 weights.  The
  * miniTE report on NVFP4 RL stability (www.aib.vote, paragraph 3) measures
@@ -428,8 +434,9 @@ size_t moe_expert_layer_w4a16_workspace_size(int64_t T, int64_t H, int64_t I,
 /* Byte offsets of the W4A16 workspace's regions: [0] error word, [1] offsets,
  * [2] padded_offsets, [3] perm, [4] inv_perm, [5] x rows (BF16, padded
  * grouped layout, zero padding rows), [6] h (BF16 [rows_cap][I]), [7] D
- * (BF16, compact sorted rows), [8..13] 0, [14] rows_cap (a count), [15] total
- * bytes.  `out` must hold 16 int64 (host memory). */
+ * (BF16, compact sorted rows), [8] h before its MXFP8 requantization (W4A8
+ * with NVFP4MOE_KEEP_H; else 0), [9..13] 0, [14] rows_cap (a count), [15]
+ * total bytes.  `out` must hold 16 int64 (host memory). */
 int moe_expert_layer_w4a16_workspace_offsets(int64_t T, int64_t H, int64_t I,
                                              int E, int k, uint32_t flags,
                                              int64_t *out);
@@ -440,6 +447,35 @@ int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx,
                            int64_t H, int64_t I, int E, int k, void *y,
                            uint32_t flags, void *workspace,
                            size_t workspace_bytes, nvfp4moe_stream_t stream);
+
+/* The MoE expert layer with NVFP4 weights and MXFP8 activations (W4A8),
+ * the third variant the same paragraph of the aib.vote report compares.  The
+ * weights are the W4A4 layer's NVFP4 weights; x (per token) and h (per row)
+ * are quantized to MXFP8 -- blocks of 32 along the row, E8M0 scale 2^s with
+ * s = floor(log2 amax) - 8, E4M3 elements, round to nearest even, saturating
+ * at +-448 (the public OCP MX definition; the pages name the format only) --
+ * and dequantized exactly.  The products then run as in
+ * moe_expert_layer_w4a16 (BF16 operands, which hold E4M3 x 2^s exactly, on
+ * the kind::f16 tensor cores with FP32 accumulation), so the result is the
+ * W4A8 layer's up to FP32 summation order.  Dequantized activations below
+ * BF16's normal range (2^-126) are rounded to BF16.
+ *   arguments  as for moe_expert_layer_w4a16
+ *   flags      0, or NVFP4MOE_KEEP_H: also keep the BF16 h before its MXFP8
+ *              requantization in workspace region [8] (BF16 [rows_cap][I])
+ *   workspace  moe_expert_layer_w4a8_workspace_size() bytes (with the same
+ *              flags); regions as for the W4A16 layer, plus [8]. */
+size_t moe_expert_layer_w4a8_workspace_size(int64_t T, int64_t H, int64_t I,
+                                            int E, int k, uint32_t flags);
+int moe_expert_layer_w4a8_workspace_offsets(int64_t T, int64_t H, int64_t I,
+                                            int E, int k, uint32_t flags,
+                                            int64_t *out);
+int moe_expert_layer_w4a8(const void *x, const int32_t *topk_idx,
+                          const float *topk_w,
+                          const nvfp4moe_weights *w_gate_up,
+                          const nvfp4moe_weights *w_down, int64_t T,
+                          int64_t H, int64_t I, int E, int k, void *y,
+                          uint32_t flags, void *workspace,
+                          size_t workspace_bytes, nvfp4moe_stream_t stream);
 
 /* ---------------------------------------------------------- diagnostics -- */
 /* The hardware conversions the quantizer uses, exposed so their rounding can

@@ -1,5 +1,6 @@
 // The C-ABI of nvfp4moe: argument checks, workspace layout and the layer's
 // launch sequence.  Plain pointers and sizes only; see include/nvfp4moe.h.
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -37,13 +38,23 @@ constexpr int64_t kHdrHAmax = 20;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
-int cuda_rc(cudaError_t e) { return e == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA; }
+// The CUDA error behind the last NVFP4MOE_ERR_CUDA of this host thread.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+thread_local int g_last_cuda_line = 0;
+
+int cuda_fail(cudaError_t e, int line) {
+  g_last_cuda_error = e;
+  g_last_cuda_line = line;
+  return NVFP4MOE_ERR_CUDA;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? NVFP4MOE_OK : cuda_fail(e, 0); }
 cudaStream_t st(nvfp4moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
-#define NVFP4MOE_TRY(expr)                 \
-  do {                                     \
-    cudaError_t e_ = (expr);               \
-    if (e_ != cudaSuccess) return NVFP4MOE_ERR_CUDA; \
+#define NVFP4MOE_TRY(expr)                              \
+  do {                                                  \
+    cudaError_t e_ = (expr);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, __LINE__); \
   } while (0)
 
 // Bump allocator over a caller-provided workspace.
@@ -141,10 +152,11 @@ BwdLayout bwd_layout(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t fla
   return L;
 }
 
-// Workspace of the W4A16 layer: [0] header, [1] offsets, [2] padded offsets,
-// [3] perm, [4] inv_perm, [5] x rows (padded), [6] h (padded), [7] D
-// (compact), [14] rows_cap, [15] total bytes.
-BwdLayout w4a16_layout(int64_t T, int64_t H, int64_t I, int E, int k) {
+// Workspace of the W4A16 / W4A8 layer: [0] header, [1] offsets, [2] padded
+// offsets, [3] perm, [4] inv_perm, [5] x rows (padded), [6] h (padded), [7] D
+// (compact), [8] h before its MXFP8 requantization (W4A8 with KEEP_H),
+// [14] rows_cap, [15] total bytes.
+BwdLayout w4a16_layout(int64_t T, int64_t H, int64_t I, int E, int k, bool keep_h_pre = false) {
   const int64_t R = T * k;
   const int64_t cap = layer_rows_cap(T, k, E);
   Carve c;
@@ -158,6 +170,7 @@ BwdLayout w4a16_layout(int64_t T, int64_t H, int64_t I, int E, int k) {
   L.v[5] = c.take(cap * H * 2);
   L.v[6] = c.take(cap * I * 2);
   L.v[7] = c.take(R * H * 2);
+  L.v[8] = keep_h_pre ? c.take(cap * I * 2) : 0;
   L.counts = c.take(permute_blocks(T) * E * 4);
   L.local_rank = c.take(R * 4);
   L.ones = 0;
@@ -178,6 +191,14 @@ int check_weights(const nvfp4moe_weights *w, int64_t E, int64_t N, int64_t K) {
 }  // namespace
 
 extern "C" {
+
+int nvfp4moe_last_cuda_error(char *buf, size_t len) {
+  if (buf != nullptr && len > 0) {
+    std::snprintf(buf, len, "%s (%s) at api.cu:%d", cudaGetErrorName(g_last_cuda_error),
+                  cudaGetErrorString(g_last_cuda_error), g_last_cuda_line);
+  }
+  return (int)g_last_cuda_error;
+}
 
 const char *nvfp4moe_status_string(int status) {
   switch (status) {
@@ -743,6 +764,7 @@ int moe_expert_layer_backward(const void *x, const int32_t *topk_idx, const floa
 
   // rows of x and dy in the padded grouped layout, row weights, ones
   BwdGatherParams gp;
+  std::memset(&gp, 0, sizeof(gp));
   gp.x = x;
   gp.dy = dy;
   gp.topk_w = topk_w;
@@ -898,28 +920,20 @@ int nvfp4moe_encode_ue4m3(const float *v, int64_t n, uint8_t *codes, nvfp4moe_st
 }
 
 
-// ------------------------------------------------------------------ W4A16 --
+// ---------------------------------------------------------- W4A16 / W4A8 --
 
-size_t moe_expert_layer_w4a16_workspace_size(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
-  (void)flags;
-  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
-  return (size_t)w4a16_layout(T, H, I, E, k).v[15];
-}
+}  // extern "C"
 
-int moe_expert_layer_w4a16_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags,
-                                             int64_t *out) {
-  (void)flags;
-  if (out == nullptr || T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
-  const BwdLayout L = w4a16_layout(T, H, I, E, k);
-  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
-  return NVFP4MOE_OK;
-}
+namespace {
 
-int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *topk_w,
-                           const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down, int64_t T, int64_t H,
-                           int64_t I, int E, int k, void *y, uint32_t flags, void *workspace, size_t workspace_bytes,
-                           nvfp4moe_stream_t stream) {
-  if (T < 0 || H <= 0 || I <= 0 || k < 1 || k > 32 || E < 1 || flags != 0) return NVFP4MOE_ERR_INVALID_ARG;
+// The W4A16 layer, or with mxfp8 the W4A8 layer (x and h MXFP8
+// quantize-dequantized in the gather and in the gate_up epilogue).
+int w4ax_layer(const void *x, const int32_t *topk_idx, const float *topk_w, const nvfp4moe_weights *w_gate_up,
+               const nvfp4moe_weights *w_down, int64_t T, int64_t H, int64_t I, int E, int k, void *y, uint32_t flags,
+               void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream, bool mxfp8) {
+  const uint32_t allowed = mxfp8 ? NVFP4MOE_KEEP_H : 0u;
+  if (T < 0 || H <= 0 || I <= 0 || k < 1 || k > 32 || E < 1 || (flags & ~allowed) != 0)
+    return NVFP4MOE_ERR_INVALID_ARG;
   if (E > 1024 || H % 256 != 0 || I % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
   int rc = check_weights(w_gate_up, E, 2 * I, H);
   if (rc != NVFP4MOE_OK) return rc;
@@ -929,7 +943,8 @@ int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *
   if (T == 0) return NVFP4MOE_OK;
   if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || y == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
-  const BwdLayout L = w4a16_layout(T, H, I, E, k);
+  const bool keep_h_pre = (flags & NVFP4MOE_KEEP_H) != 0;
+  const BwdLayout L = w4a16_layout(T, H, I, E, k, keep_h_pre);
   if (workspace == nullptr || (int64_t)workspace_bytes < L.v[15]) return NVFP4MOE_ERR_WORKSPACE;
   const int64_t cap = L.v[14];
   cudaStream_t s = st(stream);
@@ -974,6 +989,7 @@ int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *
   gp.k = k;
   gp.E = E;
   gp.x_rows = x_rows;
+  gp.mxfp8_x = mxfp8 ? 1 : 0;
   NVFP4MOE_TRY(launch_bwd_gather(gp, s));
 
   Bf16GemmArgs base;
@@ -994,6 +1010,8 @@ int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *
   g1.epilogue = kBfSwiGLUFwd;
   g1.out_bf16 = h;
   g1.out_padded = 1;
+  g1.mxfp8_h = mxfp8 ? 1 : 0;
+  g1.h_pre = keep_h_pre ? ws + L.v[8] : nullptr;
   NVFP4MOE_TRY(launch_bf16_gemm(g1, s));
   // down with NVFP4 weights -> D (compact sorted rows)
   Bf16GemmArgs g2 = base;
@@ -1009,6 +1027,54 @@ int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *
   NVFP4MOE_TRY(launch_bf16_gemm(g2, s));
   NVFP4MOE_TRY(launch_combine(d, inv_perm, topk_w, T, k, H, y, s));
   return NVFP4MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_expert_layer_w4a16_workspace_size(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
+  (void)flags;
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+  return (size_t)w4a16_layout(T, H, I, E, k).v[15];
+}
+
+int moe_expert_layer_w4a16_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags,
+                                             int64_t *out) {
+  (void)flags;
+  if (out == nullptr || T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  const BwdLayout L = w4a16_layout(T, H, I, E, k);
+  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
+  return NVFP4MOE_OK;
+}
+
+int moe_expert_layer_w4a16(const void *x, const int32_t *topk_idx, const float *topk_w,
+                           const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down, int64_t T, int64_t H,
+                           int64_t I, int E, int k, void *y, uint32_t flags, void *workspace, size_t workspace_bytes,
+                           nvfp4moe_stream_t stream) {
+  return w4ax_layer(x, topk_idx, topk_w, w_gate_up, w_down, T, H, I, E, k, y, flags, workspace, workspace_bytes,
+                    stream, false);
+}
+
+size_t moe_expert_layer_w4a8_workspace_size(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags) {
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+  return (size_t)w4a16_layout(T, H, I, E, k, (flags & NVFP4MOE_KEEP_H) != 0).v[15];
+}
+
+int moe_expert_layer_w4a8_workspace_offsets(int64_t T, int64_t H, int64_t I, int E, int k, uint32_t flags,
+                                            int64_t *out) {
+  if (out == nullptr || T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  const BwdLayout L = w4a16_layout(T, H, I, E, k, (flags & NVFP4MOE_KEEP_H) != 0);
+  for (int i = 0; i < 16; ++i) out[i] = L.v[i];
+  return NVFP4MOE_OK;
+}
+
+int moe_expert_layer_w4a8(const void *x, const int32_t *topk_idx, const float *topk_w,
+                          const nvfp4moe_weights *w_gate_up, const nvfp4moe_weights *w_down, int64_t T, int64_t H,
+                          int64_t I, int E, int k, void *y, uint32_t flags, void *workspace, size_t workspace_bytes,
+                          nvfp4moe_stream_t stream) {
+  return w4ax_layer(x, topk_idx, topk_w, w_gate_up, w_down, T, H, I, E, k, y, flags, workspace, workspace_bytes,
+                    stream, true);
 }
 
 }  // extern "C"

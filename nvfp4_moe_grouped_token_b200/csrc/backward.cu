@@ -29,8 +29,9 @@ __device__ __forceinline__ int find_group_dev(const int32_t *padded, int E, int6
 // One warp per padded row p < padded_offsets[E]: the row's token t (from the
 // permutation) gives x_rows[p] = x[t], dy_rows[p] = dy[t], w_rows[p] =
 // topk_w[t][j]; padding rows get zeros.  ones[r] = 1 for every routed row.
-// dy / dy_rows, w_rows and ones are optional (the W4A16 forward gathers x
-// alone).
+// dy / dy_rows, w_rows and ones are optional (the W4A16 / W4A8 forward
+// gathers x alone); with mxfp8_x the x rows are MXFP8 quantize-dequantized
+// (W4A8), each of the token's k rows from the same values.
 __global__ void __launch_bounds__(kGatherWarps * 32) k_bwd_gather(const BwdGatherParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
@@ -57,7 +58,33 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_bwd_gather(const BwdGathe
   uint4 *xo = static_cast<uint4 *>(p.x_rows) + row * hv;
   const uint4 z = make_uint4(0, 0, 0, 0);
   const uint4 *xs = static_cast<const uint4 *>(p.x) + (t >= 0 ? t : 0) * hv;
-  for (int64_t c = lane; c < hv; c += 32) xo[c] = t >= 0 ? __ldg(xs + c) : z;
+  if (p.mxfp8_x) {
+    // one 32-element MXFP8 block (four 16-byte chunks) per lane and step
+    for (int64_t b = lane; b < hv / 4; b += 32) {
+      if (t < 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xo[4 * b + q] = z;
+        continue;
+      }
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 u = __ldg(xs + 4 * b + q);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[8 * q + 2 * i] = bf16_lo(w[i]);
+          v[8 * q + 2 * i + 1] = bf16_hi(w[i]);
+        }
+      }
+      uint32_t o[16];
+      mxfp8_qdq32(v, o);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xo[4 * b + q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+  } else {
+    for (int64_t c = lane; c < hv; c += 32) xo[c] = t >= 0 ? __ldg(xs + c) : z;
+  }
   if (p.dy_rows != nullptr) {
     uint4 *dyo = static_cast<uint4 *>(p.dy_rows) + row * hv;
     const uint4 *dys = static_cast<const uint4 *>(p.dy) + (t >= 0 ? t : 0) * hv;

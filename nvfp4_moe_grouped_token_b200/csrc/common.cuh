@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -320,6 +321,60 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// e^-64 in binary32 (a normal number).
+constexpr float kExpM64 = 1.60381089e-28f;
+
+// silu(g) * u, the fast form g / (1 + e^-g) * u (fast exponential and
+// division, ~2^-21 relative): valid for g >= -64 (near g = -87 e^-g leaves
+// the fast division's range, 2^126, and the quotient flushes to zero).
+__device__ __forceinline__ float silu_mul_fast(float g, float u) {
+  return __fmul_rn(__fdividef(g, 1.0f + __expf(-g)), u);
+}
+
+// silu(g) * u in binary32 with one fast exponential and one fast division
+// (~2^-21 relative, far below a BF16 ulp), for every g:
+//   g >= 0:        g / (1 + e^-g) * u
+//   -64 <= g < 0:  g e^g / (1 + e^g) * u          (e^-g would overflow the
+//                                                   fast division near -87)
+//   g < -64:       ((g e^(g+64)) u) e^-64         (1 + e^g == 1 in binary32;
+//                                                   the shift keeps e^(.)
+//                                                   normal down to g = -151)
+// so silu(g) u is not flushed to zero where it is still a BF16 number.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  const bool far = g < -64.0f;
+  const float t = __expf(g >= 0.0f ? -g : (far ? g + 64.0f : g));
+  const float num = g >= 0.0f ? g : __fmul_rn(g, t);
+  const float h = __fmul_rn(__fdividef(num, far ? 1.0f : 1.0f + t), u);
+  return far ? __fmul_rn(h, kExpM64) : h;
+}
+
+// MXFP8 quantize-dequantize of one 32-element block held by one thread (the
+// public OCP MX definition; the activations of the W4A8 variant): the E8M0
+// scale is 2^s with s = floor(log2 amax) - 8, clamped to [-127, 127] (-127
+// for an all-zero block); each element becomes E4M3(v / 2^s) by the
+// hardware's round-to-nearest-even saturating conversion (sign kept), and is
+// returned as E4M3 * 2^s rounded to BF16 -- exact unless |E4M3 * 2^s| is
+// below BF16's normal range (2^-126).  v: binary32 values; out: BF16 pairs.
+__device__ __forceinline__ void mxfp8_qdq32(const float (&v)[32], uint32_t (&out)[16]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int eb = (int)(__float_as_uint(amax) >> 23);          // amax >= 0, finite
+  const int s = eb == 0 ? -127 : max(eb - 135, -127);
+  const float down = __uint_as_float((uint32_t)(127 - s) << 23);                      // 2^-s, s <= 119
+  const float up = s > -127 ? __uint_as_float((uint32_t)(s + 127) << 23) : 0x1p-127f;  // 2^s
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint16_t q;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q) : "f"(v[2 * i + 1] * down), "f"(v[2 * i] * down));
+    uint32_t hp;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hp) : "h"(q));
+    const float lo = __half2float(__ushort_as_half((unsigned short)(hp & 0xFFFFu)));
+    const float hi = __half2float(__ushort_as_half((unsigned short)(hp >> 16)));
+    out[i] = pack_bf16x2(lo * up, hi * up);
+  }
 }
 
 // Byte offset of scale (row, block b) in the MMA atom layout of a matrix whose

@@ -677,24 +677,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       if (BN == 256 && a.epilogue == kEpiSwiGLU) {
         uint32_t hp[2][16];
         float m = 0.0f;
+        auto swiglu = [&](auto silu) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float hh[2];
+            for (int i = 0; i < 32; i += 2) {
+              float hh[2];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float g = __fmul_rn(__uint_as_float(v[c][i + q]), scale);
-              const float u = __fmul_rn(__uint_as_float(v[(c + 2) % C::kChunks][i + q]), scale);
-              // silu(g) = g / (1 + e^-g); the fast exponential and division
-              // are accurate to ~2^-21 relative, far below a BF16 ulp of h
-              const float sg = __fdividef(g, 1.0f + __expf(-g));
-              hh[q] = __fmul_rn(sg, u);
+              for (int q = 0; q < 2; ++q) {
+                const float g = __fmul_rn(__uint_as_float(v[c][i + q]), scale);
+                const float u = __fmul_rn(__uint_as_float(v[(c + 2) % C::kChunks][i + q]), scale);
+                hh[q] = silu(g, u);
+              }
+              hp[c][i / 2] = pack_bf16x2(hh[0], hh[1]);
+              m = fmax_abs_bf16(m, hp[c][i / 2]);
             }
-            hp[c][i / 2] = pack_bf16x2(hh[0], hh[1]);
-            m = fmax_abs_bf16(m, hp[c][i / 2]);
           }
-        }
+        };
+        // the fast SwiGLU form unless some gate value of the warp's tile
+        // part is below -64 (scale >= 0, so the minimum decides)
+        float gmin = __uint_as_float(v[0][0]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) gmin = fminf(gmin, __uint_as_float(v[c][i]));
+        if (__any_sync(0xffffffffu, __fmul_rn(gmin, scale) < -64.0f))
+          swiglu([](float g, float u) { return silu_mul(g, u); });
+        else
+          swiglu([](float g, float u) { return silu_mul_fast(g, u); });
         // h rows live at padded positions: the whole slab is stored (rows past
         // the group's end are padding that nothing reads)
 #pragma unroll

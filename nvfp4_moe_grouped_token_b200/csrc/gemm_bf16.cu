@@ -140,11 +140,6 @@ __device__ __forceinline__ Tile tile_of(const Bf16GemmArgs &a, int64_t t, int n_
   return r;
 }
 
-__device__ __forceinline__ float silu_f(float g, float &s) {
-  s = 1.0f / (1.0f + expf(-g));
-  return g * s;
-}
-
 __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant__ BParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -401,12 +396,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
               const float g = q ? bf16_hi(gw[i]) : bf16_lo(gw[i]);
               const float u = q ? bf16_hi(uw[i]) : bf16_lo(uw[i]);
               const float dhp = __uint_as_float(v[2 * i + q]);
-              float sg;
-              const float sl = silu_f(g, sg);
-              const float h = __bfloat162float(__float2bfloat16_rn(sl * u));
               const float dh = wr * dhp;
-              dg2[q] = dh * u * (sg * (1.0f + g * (1.0f - sg)));
-              du2[q] = dh * sl;
+              // sigmoid s = sc * sp without overflow: g >= 0: sp = 1/(1+e^-g);
+              // g < 0: sp = e^g/(1+e^g); g < -64: sp = e^(g+64), sc = e^-64
+              // (then 1 + e^g and 1 - s are 1 in binary32)
+              const bool far = g < -64.0f;
+              const float t = expf(g >= 0.0f ? -g : (far ? g + 64.0f : g));
+              const float sp = g >= 0.0f ? 1.0f / (1.0f + t) : (far ? t : t / (1.0f + t));
+              const float sc = far ? kExpM64 : 1.0f;
+              const float oms = far ? 1.0f : 1.0f - sp;
+              const float gs = g * sp;
+              const float hf = (gs * u) * sc;
+              dg2[q] = (dh * u * (sp * (1.0f + g * oms))) * sc;
+              du2[q] = (dh * gs) * sc;
+              const float h = __bfloat162float(__float2bfloat16_rn(hf));
               hw2[q] = wr * h;
               dwp = __fmaf_rn(dhp, h, dwp);
             }
@@ -765,13 +768,29 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
             for (int q = 0; q < 2; ++q) {
               const float g = __fmul_rn(__uint_as_float(vg[2 * i + q]), scale);
               const float u = __fmul_rn(__uint_as_float(vu[2 * i + q]), scale);
-              // silu(g) = g / (1 + e^-g) with the fast exponential and
-              // division (~2^-21 relative, far below a BF16 ulp of h)
-              hh[q] = __fmul_rn(__fdividef(g, 1.0f + __expf(-g)), u);
+              hh[q] = silu_mul(g, u);
             }
             w16[i] = pack_bf16x2(hh[0], hh[1]);
           }
-          store_box(w16, (int32_t)(tl.n0 / 2 + half * 64 + c * 32), (int32_t)(tl.m0 + quad * 32));
+          const int32_t hcol = (int32_t)(tl.n0 / 2 + half * 64 + c * 32);
+          if (a.mxfp8_h) {
+            // W4A8: the BF16 h of these 32 columns is one MXFP8 block
+            if (a.h_pre != nullptr) {
+              uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.h_pre) +
+                                                     (tl.m0 + quad * 32 + lane) * (a.N / 2) + hcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+            }
+            float hv[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              hv[2 * i] = bf16_lo(w16[i]);
+              hv[2 * i + 1] = bf16_hi(w16[i]);
+            }
+            mxfp8_qdq32(hv, w16);
+          }
+          store_box(w16, hcol, (int32_t)(tl.m0 + quad * 32));
         }
       } else {
         const int64_t g_pad = __ldg(a.padded_offsets + tl.e);

@@ -165,6 +165,10 @@ struct Bf16GemmArgs {
   // the per-expert decode scale applied to the accumulator in the epilogue
   const uint8_t *b_sf = nullptr;
   const float *s_dec_w = nullptr;
+  // kBfSwiGLUFwd: h is MXFP8 quantize-dequantized (W4A8); h_pre (optional)
+  // receives the BF16 h before that, [rows_cap][I]
+  int mxfp8_h = 0;
+  void *h_pre = nullptr;
   int *err = nullptr;
 };
 cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s);
@@ -180,6 +184,7 @@ struct BwdGatherParams {
   int k, E;
   void *x_rows, *dy_rows;
   float *w_rows, *ones;
+  int mxfp8_x = 0;   // x rows are MXFP8 quantize-dequantized (W4A8)
 };
 cudaError_t launch_bwd_gather(const BwdGatherParams &p, cudaStream_t s);
 cudaError_t launch_bwd_dw(const float *dw_part, int64_t nparts, const int32_t *inv_perm, const int32_t *topk_idx,

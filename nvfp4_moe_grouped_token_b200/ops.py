@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4moe.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvfp4moe.h")
 
 OK = 0
+ERR_CUDA = -4
 ERR_DEVICE_TIMEOUT = -5
 ERR_DEVICE_CHECK = -7
 
@@ -82,6 +83,12 @@ _SIGS = {
                                                         ctypes.POINTER(_i64)]),
     "moe_expert_layer_w4a16": (_i32, [_vp, _vp, _vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights),
                                       _i64, _i64, _i64, _i32, _i32, _vp, _u32, _vp, _sz, _vp]),
+    "moe_expert_layer_w4a8_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32, _u32]),
+    "moe_expert_layer_w4a8_workspace_offsets": (_i32, [_i64, _i64, _i64, _i32, _i32, _u32,
+                                                       ctypes.POINTER(_i64)]),
+    "moe_expert_layer_w4a8": (_i32, [_vp, _vp, _vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights),
+                                     _i64, _i64, _i64, _i32, _i32, _vp, _u32, _vp, _sz, _vp]),
+    "nvfp4moe_last_cuda_error": (_i32, [ctypes.c_char_p, _sz]),
     "nvfp4moe_num_sms": (_i32, []),
 }
 
@@ -118,6 +125,10 @@ class NVFP4Error(RuntimeError):
 def _check(rc: int, what: str):
     if rc != OK:
         msg = lib().nvfp4moe_status_string(rc).decode()
+        if rc == ERR_CUDA:
+            buf = ctypes.create_string_buffer(256)
+            lib().nvfp4moe_last_cuda_error(buf, 256)
+            msg += ": " + buf.value.decode()
         raise NVFP4Error(f"{what}: {msg} ({rc})")
 
 
@@ -404,37 +415,59 @@ def moe_expert_layer_w4a16_workspace_size(T, H, I, E, k, flags=0) -> int:
     return int(lib().moe_expert_layer_w4a16_workspace_size(T, H, I, E, k, flags))
 
 
-_W4A16_REGIONS = ["err", "offsets", "padded_offsets", "perm", "inv_perm", "x_rows", "h", "d"]
+def moe_expert_layer_w4a8_workspace_size(T, H, I, E, k, flags=0) -> int:
+    return int(lib().moe_expert_layer_w4a8_workspace_size(T, H, I, E, k, flags))
 
 
-def moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k, flags=0) -> dict:
+_W4AX_REGIONS = ["err", "offsets", "padded_offsets", "perm", "inv_perm", "x_rows", "h", "d", "h_pre"]
+
+
+def _w4ax_offsets(fn, T, H, I, E, k, flags) -> dict:
     arr = (ctypes.c_int64 * 16)()
-    _check(lib().moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k, flags, arr),
-           "moe_expert_layer_w4a16_workspace_offsets")
-    out = {name: int(arr[i]) for i, name in enumerate(_W4A16_REGIONS)}
+    _check(getattr(lib(), fn)(T, H, I, E, k, flags, arr), fn)
+    out = {name: int(arr[i]) for i, name in enumerate(_W4AX_REGIONS)}
     out["rows_cap"] = int(arr[14])
     out["total"] = int(arr[15])
     return out
+
+
+def moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k, flags=0) -> dict:
+    return _w4ax_offsets("moe_expert_layer_w4a16_workspace_offsets", T, H, I, E, k, flags)
+
+
+def moe_expert_layer_w4a8_workspace_offsets(T, H, I, E, k, flags=0) -> dict:
+    return _w4ax_offsets("moe_expert_layer_w4a8_workspace_offsets", T, H, I, E, k, flags)
+
+
+def _w4ax_layer(fn, x, topk_idx, topk_w, w_gate_up, w_down, y, workspace, flags, stream):
+    _dev(x, topk_idx, topk_w, y, workspace)
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    I = w_down.K
+    gu, dn = w_gate_up.struct(), w_down.struct()
+    _check(getattr(lib(), fn)(_p(x), _p(topk_idx), _p(topk_w), ctypes.byref(gu), ctypes.byref(dn), T, H, I,
+                              w_down.E, k, _p(y), flags, _p(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)), fn)
 
 
 def moe_expert_layer_w4a16(x, topk_idx, topk_w, w_gate_up: NVFP4Weights, w_down: NVFP4Weights, y,
                            workspace, flags=0, stream=None):
     """moe_expert_layer_w4a16: BF16 activations, the same prepared NVFP4
     weights as moe_expert_layer."""
-    _dev(x, topk_idx, topk_w, y, workspace)
-    T, H = x.shape
-    k = topk_idx.shape[1]
-    I = w_down.K
-    gu, dn = w_gate_up.struct(), w_down.struct()
-    _check(lib().moe_expert_layer_w4a16(_p(x), _p(topk_idx), _p(topk_w), ctypes.byref(gu), ctypes.byref(dn),
-                                        T, H, I, w_down.E, k, _p(y), flags, _p(workspace),
-                                        workspace.numel() * workspace.element_size(), _stream(stream)),
-           "moe_expert_layer_w4a16")
+    _w4ax_layer("moe_expert_layer_w4a16", x, topk_idx, topk_w, w_gate_up, w_down, y, workspace, flags, stream)
 
 
-def w4a16_views(workspace: torch.Tensor, T, H, I, E, k) -> dict:
-    """Typed views of the W4A16 workspace's regions (for inspection in tests)."""
-    o = moe_expert_layer_w4a16_workspace_offsets(T, H, I, E, k)
+def moe_expert_layer_w4a8(x, topk_idx, topk_w, w_gate_up: NVFP4Weights, w_down: NVFP4Weights, y,
+                          workspace, flags=0, stream=None):
+    """moe_expert_layer_w4a8: MXFP8 activations (x and h), the same prepared
+    NVFP4 weights as moe_expert_layer; flags 0 or KEEP_H."""
+    _w4ax_layer("moe_expert_layer_w4a8", x, topk_idx, topk_w, w_gate_up, w_down, y, workspace, flags, stream)
+
+
+def w4a16_views(workspace: torch.Tensor, T, H, I, E, k, flags=0, w4a8=False) -> dict:
+    """Typed views of the W4A16 / W4A8 workspace's regions (for inspection in tests)."""
+    o = (moe_expert_layer_w4a8_workspace_offsets if w4a8 else moe_expert_layer_w4a16_workspace_offsets)(
+        T, H, I, E, k, flags)
     cap = o["rows_cap"]
     R = T * k
     ws = workspace
@@ -442,7 +475,7 @@ def w4a16_views(workspace: torch.Tensor, T, H, I, E, k) -> dict:
     def view(name, nbytes, dtype, shape):
         return ws[o[name]:o[name] + nbytes].view(dtype).view(*shape)
 
-    return {
+    v = {
         "rows_cap": cap,
         "offsets": view("offsets", (E + 1) * 4, torch.int32, (E + 1,)),
         "padded_offsets": view("padded_offsets", (E + 1) * 4, torch.int32, (E + 1,)),
@@ -452,6 +485,9 @@ def w4a16_views(workspace: torch.Tensor, T, H, I, E, k) -> dict:
         "h": view("h", cap * I * 2, torch.bfloat16, (cap, I)),
         "d": view("d", R * H * 2, torch.bfloat16, (R, H)),
     }
+    if w4a8 and flags & KEEP_H:
+        v["h_pre"] = view("h_pre", cap * I * 2, torch.bfloat16, (cap, I))
+    return v
 
 
 def nvfp4moe_encode_e2m1(y: torch.Tensor, codes: torch.Tensor, stream=None):

@@ -193,6 +193,19 @@ def test_backward_with_empty_experts_and_ragged_groups():
     b.end_to_end()
 
 
+def test_backward_wide_row_scales():
+    """Rows of x scaled by 2^-20 .. 2^20: G reaches far below -64, where the
+    sigmoid's e^-g overflows binary32; dG, w*h and the <dh', h> partials must
+    still match the exact SwiGLU backward of the GPU's own G."""
+    b = Bwd(SMALL)
+    g = torch.Generator().manual_seed(13)
+    sc = torch.exp2(torch.randint(-20, 21, (SMALL.T, 1), generator=g).float())
+    b.inp["x"] = (b.inp["x"].float() * sc).to(torch.bfloat16)
+    b.d["x"] = b.inp["x"].cuda()
+    b.run()
+    b.check()
+
+
 def test_backward_without_keep_dh_matches():
     """The debug copy of dh' changes nothing else."""
     a = Bwd(SMALL)

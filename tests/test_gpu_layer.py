@@ -132,6 +132,20 @@ def test_small_layer_all_rows(flags):
     L.check()
 
 
+def test_small_layer_wide_row_scales():
+    """Rows of x scaled by 2^-20 .. 2^20 (the per-token scales follow them):
+    G reaches far below -64, where e^-g would overflow the fast division in
+    a plain g / (1 + e^-g); h must still be within tolerance of the exact
+    silu(g) u, which is a BF16 number down to g ~ -100."""
+    L = Layer(SMALL, ops.STRICT)
+    g = torch.Generator().manual_seed(12)
+    sc = torch.exp2(torch.randint(-20, 21, (SMALL.T, 1), generator=g).float())
+    L.inp["x"] = (L.inp["x"].float() * sc).to(torch.bfloat16)
+    L.x = L.inp["x"].cuda()
+    L.run()
+    L.check(check_weights=False)
+
+
 def test_small_layer_end_to_end_against_full_oracle():
     L = Layer(SMALL, ops.STRICT)
     L.run()
