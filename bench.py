@@ -56,6 +56,8 @@ def parse():
                     help="extra workloads measured at one GPU and reported under 'workloads' ('' = none)")
     ap.add_argument("--workload-steps", type=int, default=20)
     ap.add_argument("--no-backward", action="store_true", help="skip timing the BF16 backward")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip timing the W4A16 and W4A8 activation-precision variants")
     ap.add_argument("--no-fast-combine", action="store_true",
                     help="skip measuring the non-strict (FP32-reduction) combine beside the headline")
     return ap.parse_args()
@@ -441,6 +443,50 @@ def measure_backward(cfg, dev, steps, warmup):
             "note": "BF16-backward mode: exact gradient of the unquantized layer on BF16 operands (gate_up recomputed)"}
 
 
+def measure_variant(cfg, dev, steps, warmup, kind):
+    """Time the W4A16 or W4A8 layer (NVFP4 weights; BF16 or MXFP8
+    activations, products on the BF16 tensor cores) on the workload, inputs
+    resident in HBM, outside the headline's timed region.  The rate reported
+    is the layer's GEMM FLOPs over the whole step time (routing, gather, both
+    GEMMs and the combine), against the BF16 peak; the GEMM's own share of
+    the step is in the ncu launch list under profiles/."""
+    from nvfp4_moe_grouped_token_b200 import ops
+
+    inp = workloads.layer_inputs(cfg)
+    x, idx, w = inp["x"].to(dev), inp["topk_idx"].to(dev), inp["topk_w"].to(dev)
+    wgu = ops.nvfp4_prepare_weights(inp["w_gate_up"].to(dev), gate_up=True)
+    wdn = ops.nvfp4_prepare_weights(inp["w_down"].to(dev), gate_up=False)
+    size = ops.moe_expert_layer_w4a8_workspace_size if kind == "w4a8" else ops.moe_expert_layer_w4a16_workspace_size
+    call = ops.moe_expert_layer_w4a8 if kind == "w4a8" else ops.moe_expert_layer_w4a16
+    ws = torch.empty(size(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k), dtype=torch.uint8, device=dev)
+    y = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        call(x, idx, w, wgu, wdn, y, ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ops.device_status(ws) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert ops.device_status(ws) == 0
+    ms = e0.elapsed_time(e1) / steps
+    fl = layer_flops(cfg)["total"]
+    pk = peaks()
+    tf = fl / (ms * 1e-3) / 1e12
+    act = "MXFP8 (E4M3, E8M0 per 32)" if kind == "w4a8" else "BF16"
+    return {"ms_per_step": ms, "tokens_per_s": cfg.T / (ms * 1e-3), "tflops": tf, "flop": fl,
+            "frac_bf16_burst": tf / pk["bf16_tflops"], "bf16_peak": pk["bf16_tflops"], "bf16_source": pk["source"],
+            "steps": steps, "activations": act, "weights": "NVFP4 (the headline's prepared weights)",
+            "note": "weights stay 4-bit in HBM and are converted to BF16 per K-step in shared memory; "
+                    "kind::f16 tensor cores; the whole step (routing, gather, both GEMMs, combine) is timed"}
+
+
 WORKLOAD_NAMES = {
     "toy": "toy NVFP4 MoE layer (E=4, T=256, top-2, K=256 -> N=512)",
     "dense4b": "dense Qwen3-4B-shaped W4A4 MLP (T=8192, 2560 -> 2x9728 -> 2560, 0.1% outlier channels x30)",
@@ -503,6 +549,11 @@ def run_ours(args, rank, world, local_rank):
                                            "(bitwise the same outputs); off by default because it is slower"}
     if world == 1 and not args.no_backward:
         result["backward"] = measure_backward(cfg, dev, max(5, args.steps // 5), 2)
+        torch.cuda.empty_cache()
+    if world == 1 and not args.no_variants:
+        for kind in ("w4a16", "w4a8"):
+            result[kind] = measure_variant(cfg, dev, max(5, args.steps // 5), 3, kind)
+            torch.cuda.empty_cache()
         torch.cuda.empty_cache()
     if world == 1 and args.workloads:
         extra = {}

@@ -462,27 +462,79 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
 // factor is a BF16 subnormal for subnormal UE4M3 scales, which the BF16
 // multiply keeps.)
 //
-//   raw ring (4 stages): A 16 KB (TMA, swizzled) + codes 8 KB (TMA, 256 rows
-//     x 32 bytes, unswizzled) + scales 1 KB (two 512-byte atoms, bulk copies)
-//   converted ring (2 slots): B as BF16, 32 KB each
+// The conversion is the expensive part (about as many issue slots as the
+// MMAs take time for a 128 x 256 tile), so each converted weight tile feeds
+// two m-tiles of the same expert: a unit is (m-tile pair, 128 weight rows),
+// two M = 128, N = 128 MMAs per K-slice share the B operand, and the
+// conversion per FLOP halves.  An expert with an odd number of m-tiles ends
+// with a single-m-tile unit.  For the gate_up weight (rows interleaved in
+// blocks of 128 gate then 128 up) a unit's 128 rows are 64 gate rows and the
+// 64 matching up rows, so the SwiGLU epilogue finds both in one tile.
+//
+//   raw ring (4 stages): A of both m-tiles 2 x 16 KB (TMA, swizzled) +
+//     codes 4 KB (two TMA boxes of 64 rows x 32 bytes, unswizzled) + scales
+//     1 KB (the two 512-byte atoms holding those rows, bulk copies)
+//   converted ring (2 slots): B as BF16, 16 KB each
+//   TMEM: two buffers of 2 x 128 accumulator columns (epilogue of one unit
+//     overlaps the MMAs of the next)
 //   warp 0: producer; warp 1: TMEM owner + MMA issuer; warps 2-9: epilogue
-//   (two per TMEM lane quarter); warps 10-17: converters, four rows' halves
-//   per lane and K-step.
+//   (m-tile = which half of the warps, TMEM lane quarter = warp % 4);
+//   warps 10-17: converters, one half row per lane and K-step.
 namespace w4 {
 constexpr int RS = 4;
 constexpr int CS = 2;
-constexpr int kCodesBytes = BN * BK / 2;                  // 8 KB
-constexpr int kSfBytes = BN * BK / 16;                    // 1 KB
-constexpr int kRawBytes = kABytes + kCodesBytes + kSfBytes;
+constexpr int WN = 128;                                   // weight rows per unit
+constexpr int kA2Bytes = 2 * kABytes;                     // A of two m-tiles
+constexpr int kCodesBytes = WN * BK / 2;                  // 4 KB
+constexpr int kSfBytes = 2 * 512;                         // two scale atoms
+constexpr int kRawBytes = kA2Bytes + kCodesBytes + kSfBytes;
+constexpr int kConvBytes = WN * BK * 2;                   // 16 KB
+constexpr int kAccCols = 2 * WN;                          // one buffer: two m-tiles
 constexpr int kThreads = 576;
 constexpr int kEpiWarp0 = 2, kConvWarp0 = 10, kConvWarps = 8;
 constexpr size_t kConvOff = (size_t)RS * kRawBytes;
-constexpr size_t kStagingOff = kConvOff + (size_t)CS * kBBytes;
+constexpr size_t kStagingOff = kConvOff + (size_t)CS * kConvBytes;
 constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
-constexpr size_t kSmemBytes = kBarrierOff + 256 + 1024;
-static_assert(kRawBytes % 1024 == 0 && kBBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kConvWarps * 32 * 2 == 2 * BN, "each converter lane covers two half rows");
+constexpr size_t kPairsOff = kBarrierOff + 256;           // + (E + 1) int32 pair prefix
+constexpr size_t kSmemMax = kPairsOff + 4 * 1025 + 1024;  // + up to 1023 bytes of alignment
+static_assert(kRawBytes % 1024 == 0 && kConvBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+static_assert(kSmemMax <= 232448, "shared memory budget");
+static_assert(kConvWarps * 32 == 2 * WN, "each converter lane covers one half row");
+static_assert(ACC * kAccCols <= 512, "TMEM budget");
+// Instruction descriptor as idesc_bf16 with N = 128, both operands K-major.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(WN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+// A unit's m-tiles and weight rows.
+struct Unit {
+  int e;
+  int64_t m0;       // first padded row of the first m-tile
+  bool two;         // a second m-tile at m0 + 128
+  int nt;           // weight-row tile
+  int64_t wrow0;    // first weight row of each 64-row half (global row of the [E*N] codes)
+  int64_t wrow1;
+};
+
+__device__ __forceinline__ Unit unit_of(const Bf16GemmArgs &a, const int32_t *pairs, int64_t u, int n_tiles,
+                                        int64_t rows_cap) {
+  Unit r;
+  const int64_t p = u / n_tiles;
+  r.nt = (int)(u - p * n_tiles);
+  int lo = 0, hi = a.E;                    // the expert whose pairs hold p
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)pairs[mid] <= p) lo = mid; else hi = mid;
+  }
+  r.e = lo;
+  const int64_t g_lo = min((int64_t)__ldg(a.padded_offsets + lo), rows_cap);
+  const int64_t g_hi = min((int64_t)__ldg(a.padded_offsets + lo + 1), rows_cap);
+  r.m0 = g_lo + 2 * BM * (p - pairs[lo]);
+  r.two = r.m0 + BM < g_hi;
+  const bool gate_up = a.epilogue == kBfSwiGLUFwd;
+  r.wrow0 = (int64_t)r.e * a.N + (gate_up ? 256 * (r.nt >> 1) + 64 * (r.nt & 1) : (int64_t)WN * r.nt);
+  r.wrow1 = r.wrow0 + (gate_up ? 128 : 64);
+  return r;
+}
 }  // namespace w4
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -557,6 +609,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *never = reinterpret_cast<int *>(tmem_slot + 2);
+  int32_t *pairs = reinterpret_cast<int32_t *>(smem + kPairsOff);   // [E + 1]
 
   const Bf16GemmArgs &a = P.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -587,16 +640,35 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (warp == 2) {
+    // pairs[e] = m-tile pairs of the experts before e (groups clipped to rows_cap)
+    int32_t carry = 0;
+    if (lane == 0) pairs[0] = 0;
+    for (int base = 0; base < a.E; base += 32) {
+      const int e = base + lane;
+      int32_t n = 0;
+      if (e < a.E) {
+        const int64_t lo = min((int64_t)__ldg(a.padded_offsets + e), a.rows_cap);
+        const int64_t hi = min((int64_t)__ldg(a.padded_offsets + e + 1), a.rows_cap);
+        const int64_t tiles = hi > lo ? (hi - lo) / BM : 0;
+        n = (int32_t)((tiles + 1) / 2);
+      }
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, n, o);
+        if (lane >= o) n += v;
+      }
+      if (e < a.E) pairs[e + 1] = carry + n;
+      carry += __shfl_sync(0xffffffffu, n, 31);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int n_tiles = (int)(a.N / BN);
-  int64_t rows_used = __ldg(a.padded_offsets + a.E);
-  if (rows_used > a.rows_cap) rows_used = a.rows_cap;
-  if (rows_used < 0) rows_used = 0;
-  const int64_t total = (rows_used / BM) * n_tiles;
+  const int n_tiles = (int)(a.N / WN);
+  const int64_t total = (int64_t)pairs[a.E] * n_tiles;
   const int ksteps = (int)(a.K / BK);
   const int64_t k_atoms = a.K >> 6;
 
@@ -606,18 +678,21 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
       uint32_t p = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = tile_of(a, t, n_tiles, 0);
-        const int64_t wrow = (int64_t)tl.e * a.N + tl.n0;
-        const uint8_t *sf0 = a.b_sf + (wrow >> 7) * k_atoms * 512;
+        const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
+        const uint8_t *sf0 = a.b_sf + (un.wrow0 >> 7) * k_atoms * 512;
+        const uint8_t *sf1 = a.b_sf + (un.wrow1 >> 7) * k_atoms * 512;
+        const uint32_t bytes = un.two ? kRawBytes : kRawBytes - kABytes;
         uint32_t st = p % RS, ph = (p / RS) & 1u;
         for (int kt = 0; kt < ksteps; ++kt, ++p) {
           if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, a.err, 530)) { ok = false; break; }
           uint8_t *raw = smem + (size_t)st * kRawBytes;
-          mbar_arrive_expect_tx(&full[st], kRawBytes);
-          tma_load_2d(raw, &P.tmap_a, kt * BK, (int32_t)tl.m0, &full[st]);
-          tma_load_2d(raw + kABytes, &P.tmap_b, kt * (BK / 2), (int32_t)wrow, &full[st]);
-          bulk_load(raw + kABytes + kCodesBytes, sf0 + (int64_t)kt * 512, 512, &full[st]);
-          bulk_load(raw + kABytes + kCodesBytes + 512, sf0 + (k_atoms + kt) * 512, 512, &full[st]);
+          mbar_arrive_expect_tx(&full[st], bytes);
+          tma_load_2d(raw, &P.tmap_a, kt * BK, (int32_t)un.m0, &full[st]);
+          if (un.two) tma_load_2d(raw + kABytes, &P.tmap_a, kt * BK, (int32_t)(un.m0 + BM), &full[st]);
+          tma_load_2d(raw + kA2Bytes, &P.tmap_b, kt * (BK / 2), (int32_t)un.wrow0, &full[st]);
+          tma_load_2d(raw + kA2Bytes + kCodesBytes / 2, &P.tmap_b, kt * (BK / 2), (int32_t)un.wrow1, &full[st]);
+          bulk_load(raw + kA2Bytes + kCodesBytes, sf0 + (int64_t)kt * 512, 512, &full[st]);
+          bulk_load(raw + kA2Bytes + kCodesBytes + 512, sf1 + (int64_t)kt * 512, 512, &full[st]);
           if (++st == RS) { st = 0; ph ^= 1u; }
         }
       }
@@ -628,13 +703,13 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer
       const uint64_t dk = smem_desc(0, 16, 1024, 2);
-      const uint32_t idesc = idesc_bf16(0, 0);
       const uint32_t smem0 = smem_u32(smem);
       uint32_t p = 0, it = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
         const uint32_t as = it % ACC;
-        const uint32_t acc = tmem + as * BN;
+        const uint32_t acc = tmem + as * kAccCols;
         if (!mbar_wait_bounded(&acc_empty[as], ((it / ACC) & 1u) ^ 1u, abort_flag, a.err, 540)) break;
         tc_fence_after();
         for (int kt = 0; kt < ksteps; ++kt, ++p) {
@@ -646,10 +721,13 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
           }
           tc_fence_after();
           const uint64_t a16 = (smem0 + st * (uint32_t)kRawBytes) >> 4;
-          const uint64_t b16 = (smem0 + (uint32_t)kConvOff + cs * (uint32_t)kBBytes) >> 4;
+          const uint64_t b16 = (smem0 + (uint32_t)kConvOff + cs * (uint32_t)kConvBytes) >> 4;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16(acc, dk | (a16 + kk * 2), dk | (b16 + kk * 2), idesc, (kt | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t accum = (kt | kk) != 0 ? 1u : 0u;
+            mma_bf16(acc, dk | (a16 + kk * 2), dk | (b16 + kk * 2), kIdesc, accum);
+            if (un.two) mma_bf16(acc + WN, dk | (a16 + kABytes / 16 + kk * 2), dk | (b16 + kk * 2), kIdesc, accum);
+          }
           tc_commit(&empty[st]);
           tc_commit(&cempty[cs]);
         }
@@ -660,26 +738,28 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     }
   } else if (warp >= kConvWarp0) {
     // ------------------------------------------------------- converters
-    // Lane l of converter warp w covers K-half (l & 1) of B rows
-    // 32w + l/2 and 32w + 16 + l/2: its 16-byte code loads are contiguous
-    // across the warp, and its 16-byte stores land in distinct banks within
-    // every quarter warp under the 128-byte swizzle.
+    // Lane l of converter warp w covers K-half (l & 1) of B row
+    // r = 16w + l/2 (rows 0-63 from the first 64-row box, 64-127 from the
+    // second): its 16-byte code loads are contiguous across the warp, and its
+    // 16-byte stores land in distinct banks within every quarter warp under
+    // the 128-byte swizzle.
     const int cw = warp - kConvWarp0;
     const int hk = lane & 1;
+    const int r = 16 * cw + (lane >> 1);
+    const int half_box = r >> 6;
     const uint32_t smem0 = smem_u32(smem);
-    uint32_t code_off[2], sf_off[2], dst_off[2][4];
+    const uint32_t code_off = (uint32_t)(kA2Bytes + r * 32 + hk * 16);
+    uint32_t dst_off[4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int r = 32 * cw + 16 * j + (lane >> 1);
-      code_off[j] = (uint32_t)(kABytes + r * 32 + hk * 16);
-      sf_off[j] = (uint32_t)(kABytes + kCodesBytes + (r >> 7) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + 2 * hk);
-      // 16-byte chunk 4hk + i of row r under the 128-byte swizzle
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst_off[j][i] = (uint32_t)(r * 128) + ((uint32_t)((4 * hk + i) ^ (r & 7)) << 4);
-    }
+    for (int i = 0; i < 4; ++i) dst_off[i] = (uint32_t)(r * 128) + ((uint32_t)((4 * hk + i) ^ (r & 7)) << 4);
     uint32_t p = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
+      // the row's place in its 128-row scale atom
+      const int ra = (int)(((half_box ? un.wrow1 : un.wrow0) & 127) + (r & 63));
+      const uint32_t sf_off = (uint32_t)(kA2Bytes + kCodesBytes + half_box * 512 + (ra & 31) * 16 + (ra >> 5) * 4 +
+                                         2 * hk);
       for (int kt = 0; kt < ksteps; ++kt, ++p) {
         const uint32_t st = p % RS, cs = p % CS;
         if (!mbar_wait_bounded(&full[st], (p / RS) & 1u, abort_flag, a.err, 550) ||
@@ -688,27 +768,19 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
           break;
         }
         const uint32_t raw = smem0 + st * (uint32_t)kRawBytes;
-        const uint32_t dst = smem0 + (uint32_t)kConvOff + cs * (uint32_t)kBBytes;
-        uint4 q[2];
-        uint32_t sc[2];
+        const uint32_t dst = smem0 + (uint32_t)kConvOff + cs * (uint32_t)kConvBytes;
+        const uint4 q = ld_shared_v4(raw + code_off);
+        const uint32_t sc = ld_shared_u16(raw + sf_off);
+        uint32_t s2[2];
+        ue4m3x2_to_bf16x2(sc, s2[0], s2[1]);
+        const uint32_t cw4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          q[j] = ld_shared_v4(raw + code_off[j]);
-          sc[j] = ld_shared_u16(raw + sf_off[j]);
-        }
+        for (int i = 0; i < 4; ++i) {
+          uint32_t w[4];
+          e2m1x8_to_bf16x2(cw4[i], w);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t s2[2];
-          ue4m3x2_to_bf16x2(sc[j], s2[0], s2[1]);
-          const uint32_t cw4[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t w[4];
-            e2m1x8_to_bf16x2(cw4[i], w);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) w[u] = mul_bf16x2(w[u], s2[i >> 1]);
-            st_shared_v4(dst + dst_off[j][i], w[0], w[1], w[2], w[3]);
-          }
+          for (int u = 0; u < 4; ++u) w[u] = mul_bf16x2(w[u], s2[i >> 1]);
+          st_shared_v4(dst + dst_off[i], w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -719,7 +791,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     // -------------------------------------------------------- epilogue
     const int ew = warp - w4::kEpiWarp0;
     const int quad = warp & 3;
-    const int half = ew >> 2;
+    const int half = ew >> 2;              // which m-tile of the unit
     const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
     uint8_t *stg = smem + w4::kStagingOff + (size_t)ew * kStagingPerWarp;
     const uint32_t stg_addr = smem_u32(stg);
@@ -737,47 +809,50 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
       }
       ++chunk_id;
     };
+    auto release = [&](uint32_t as) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[as]);
+    };
     const int64_t rows_total = (int64_t)__ldg(a.offsets + a.E);
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const Tile tl = tile_of(a, t, n_tiles, 0);
+      const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
       const uint32_t as = it % ACC;
-      const float scale = __ldg(a.s_dec_w + tl.e);
+      const float scale = __ldg(a.s_dec_w + un.e);
       if (!mbar_wait_bounded(&acc_full[as], (it / ACC) & 1u, abort_flag, a.err, 560)) break;
       tc_fence_after();
-      const uint32_t tacc = tlane + as * BN;
+      if (half == 1 && !un.two) {            // a single-m-tile unit
+        release(as);
+        continue;
+      }
+      const uint32_t tacc = tlane + as * kAccCols + half * WN;
+      const int64_t mrow0 = un.m0 + half * BM;
       if (a.epilogue == kBfSwiGLUFwd) {
-        // gate columns [half*64, +64), up columns [128 + half*64, +64) of the
-        // tile (the gate_up weight rows are interleaved in blocks of 128);
-        // h columns n0/2 + half*64 + [0, 64), every padded row of the slab
+        // gate columns [0, 64), up columns [64, 128) of the unit; h columns
+        // 64 nt + [0, 64), every padded row of the slab
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t vg[32], vu[32];
-          tmem_ld_32cols(tacc + half * 64 + c * 32, vg);
-          tmem_ld_32cols(tacc + 128 + half * 64 + c * 32, vu);
+          tmem_ld_32cols(tacc + c * 32, vg);
+          tmem_ld_32cols(tacc + 64 + c * 32, vu);
           tmem_ld_wait();
-          if (c == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[as]);
-          }
+          if (c == 1) release(as);
           uint32_t w16[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             float hh[2];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float g = __fmul_rn(__uint_as_float(vg[2 * i + q]), scale);
-              const float u = __fmul_rn(__uint_as_float(vu[2 * i + q]), scale);
-              hh[q] = silu_mul(g, u);
-            }
+            for (int q = 0; q < 2; ++q)
+              hh[q] = silu_mul(__fmul_rn(__uint_as_float(vg[2 * i + q]), scale),
+                               __fmul_rn(__uint_as_float(vu[2 * i + q]), scale));
             w16[i] = pack_bf16x2(hh[0], hh[1]);
           }
-          const int32_t hcol = (int32_t)(tl.n0 / 2 + half * 64 + c * 32);
+          const int32_t hcol = (int32_t)(64 * un.nt + c * 32);
           if (a.mxfp8_h) {
             // W4A8: the BF16 h of these 32 columns is one MXFP8 block
             if (a.h_pre != nullptr) {
               uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.h_pre) +
-                                                     (tl.m0 + quad * 32 + lane) * (a.N / 2) + hcol);
+                                                     (mrow0 + quad * 32 + lane) * (a.N / 2) + hcol);
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
@@ -790,29 +865,25 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
             }
             mxfp8_qdq32(hv, w16);
           }
-          store_box(w16, hcol, (int32_t)(tl.m0 + quad * 32));
+          store_box(w16, hcol, (int32_t)(mrow0 + quad * 32));
         }
       } else {
-        const int64_t g_pad = __ldg(a.padded_offsets + tl.e);
-        const int64_t g_off = __ldg(a.offsets + tl.e);
-        const int64_t g_cnt = (int64_t)__ldg(a.offsets + tl.e + 1) - g_off;
-        const int64_t rel = tl.m0 - g_pad + quad * 32 + lane;
+        const int64_t g_pad = __ldg(a.padded_offsets + un.e);
+        const int64_t g_off = __ldg(a.offsets + un.e);
+        const int64_t g_cnt = (int64_t)__ldg(a.offsets + un.e + 1) - g_off;
+        const int64_t rel = mrow0 - g_pad + quad * 32 + lane;
         const bool valid = rel < g_cnt && g_off + rel < rows_total;
-        const int64_t prow = tl.m0 + quad * 32 + lane;
+        const int64_t prow = mrow0 + quad * 32 + lane;
         const int64_t orow = a.out_padded ? prow : g_off + rel;
-        const bool slab_full = a.out_padded || (tl.m0 - g_pad) + quad * 32 + 32 <= g_cnt;
-        const int64_t slab_row = a.out_padded ? tl.m0 + quad * 32 : g_off + (tl.m0 - g_pad) + quad * 32;
-        const int64_t col0 = tl.n0 + half * 128;
+        const bool slab_full = a.out_padded || (mrow0 - g_pad) + quad * 32 + 32 <= g_cnt;
+        const int64_t slab_row = a.out_padded ? mrow0 + quad * 32 : g_off + (mrow0 - g_pad) + quad * 32;
+        const int64_t col0 = (int64_t)WN * un.nt;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
-          tmem_ld_32cols(tacc + half * 128 + c * 32, v);
+          tmem_ld_32cols(tacc + c * 32, v);
           tmem_ld_wait();
-          if (c == 3) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[as]);
-          }
+          if (c == 3) release(as);
           uint32_t w16[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -845,14 +916,15 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
 
 static cudaError_t launch_w4a16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
   if (a.mode != kBfRows || a.b_mn || a.s_dec_w == nullptr || a.out_bf16 == nullptr || a.K % BK != 0 ||
-      (a.epilogue != kBfStore && a.epilogue != kBfSwiGLUFwd) || (a.epilogue == kBfSwiGLUFwd && !a.out_padded))
+      a.E < 1 || a.E > 1024 || (a.epilogue != kBfStore && a.epilogue != kBfSwiGLUFwd) ||
+      (a.epilogue == kBfSwiGLUFwd && (!a.out_padded || a.N % 256 != 0)) || a.N % w4::WN != 0)
     return cudaErrorInvalidValue;
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (configured_device != dev) {
-    err = cudaFuncSetAttribute(k_w4a16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)w4::kSmemBytes);
+    err = cudaFuncSetAttribute(k_w4a16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)w4::kSmemMax);
     if (err != cudaSuccess) return err;
     configured_device = dev;
   }
@@ -861,18 +933,21 @@ static cudaError_t launch_w4a16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.K, (uint64_t)a.rows_cap, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  // weight codes: boxes of 64 rows x 32 bytes (one K-step of half a unit)
   if (!encode_2d_map(&P.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b, (uint64_t)(a.K / 2), (uint64_t)(a.E * a.N),
-                     BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     BK / 2, w4::WN / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const uint64_t out_cols = a.epilogue == kBfSwiGLUFwd ? (uint64_t)(a.N / 2) : (uint64_t)a.N;
   if (!encode_2d_map(&P.tmap_out, BF, 2, a.out_bf16, out_cols, (uint64_t)a.rows_cap, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  const int64_t tiles = (a.rows_cap / BM) * (a.N / BN);
+  // units: at most (m-tiles + experts) / 2 pairs times the weight-row tiles
+  const int64_t units = ((a.rows_cap / BM + a.E) / 2 + 1) * (a.N / w4::WN);
   int64_t grid = num_sms();
-  if (grid > tiles) grid = tiles;
+  if (grid > units) grid = units;
   if (grid < 1) grid = 1;
-  k_w4a16_gemm<<<(unsigned)grid, w4::kThreads, w4::kSmemBytes, s>>>(P);
+  const size_t smem = w4::kPairsOff + 4 * (size_t)(a.E + 1) + 1024;
+  k_w4a16_gemm<<<(unsigned)grid, w4::kThreads, smem, s>>>(P);
   return cudaGetLastError();
 }
 
