@@ -763,8 +763,7 @@ int moe_expert_layer_backward(const void *x, const int32_t *topk_idx, const floa
   NVFP4MOE_TRY(launch_route_rank(pp, s));
 
   // rows of x and dy in the padded grouped layout, row weights, ones
-  BwdGatherParams gp;
-  std::memset(&gp, 0, sizeof(gp));
+  BwdGatherParams gp{};
   gp.x = x;
   gp.dy = dy;
   gp.topk_w = topk_w;
@@ -975,8 +974,7 @@ int w4ax_layer(const void *x, const int32_t *topk_idx, const float *topk_w, cons
   NVFP4MOE_TRY(launch_route_count(pp, s));
   NVFP4MOE_TRY(launch_route_scan(pp, s));
   NVFP4MOE_TRY(launch_route_rank(pp, s));
-  BwdGatherParams gp;
-  std::memset(&gp, 0, sizeof(gp));
+  BwdGatherParams gp{};
   gp.x = x;
   gp.topk_w = topk_w;
   gp.topk_idx = topk_idx;
