@@ -84,11 +84,15 @@ constexpr int kSlabRows = 32;
 // pieces in flight per warp.
 constexpr uint32_t kReqPiece = 5632;
 
-template <int BN_, int STAGES_, int ACC_>
+template <int BN_, int STAGES_, int ACC_, bool SWIGLU_>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr int STAGES = STAGES_;
   static constexpr int ACC = ACC_;                   // TMEM accumulator buffers
+  // the epilogue this instantiation carries: SwiGLU (gate_up) or the plain
+  // store / FP32 reduction (down); compiling only one keeps the other's
+  // registers out of the kernel
+  static constexpr bool SWIGLU = SWIGLU_;
   static constexpr int kABytes = BM * BK / 2;        // 16 KB of E2M1 codes
   static constexpr int kBBytes = BN * BK / 2;
   static constexpr int kSfaBytes = BM * BK / 16;     // four 512-byte atoms
@@ -118,8 +122,8 @@ struct Cfg {
   static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 12 <= 192, "pipeline barriers overrun their area");
 };
 
-using CfgGateUp = Cfg<256, 3, 1>;
-using CfgDown = Cfg<256, 3, 1>;
+using CfgGateUp = Cfg<256, 3, 1, true>;
+using CfgDown = Cfg<256, 3, 1, false>;
 
 struct __align__(64) KParams {
   CUtensorMap tmap_a;
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   const GemmArgs &a = P.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // requantize h inside this launch (SwiGLU epilogue, per-row amax)
-  const bool fused_requant = a.epilogue == kEpiSwiGLU && a.req_q != nullptr && a.amax_h != nullptr &&
+  const bool fused_requant = C::SWIGLU && a.req_q != nullptr && a.amax_h != nullptr &&
                              a.amax_h_rows != 0;
 
   if (threadIdx.x == 0) {
@@ -639,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       tc_fence_after();
       uint32_t v[C::kChunks][32];
       const uint32_t tacc = tlane + as * BN;
-      if (a.epilogue == kEpiSwiGLU) {
+      if constexpr (C::SWIGLU) {
         // gate columns [half*64, +64) and up columns [128 + half*64, +64)
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
@@ -656,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       const float scale = __fmul_rn(sa, sw);
       // rows of this warp's 32-row slab all belong to the group?
       const bool slab_full = (row0 - g_pad) + quad * 32 + 32 <= g_cnt;
-      if (BN == 256 && a.epilogue == kEpiSwiGLU) {
+      if constexpr (C::SWIGLU) {
         uint32_t hp[2][16];
         float m = 0.0f;
         auto swiglu = [&](auto silu) {
