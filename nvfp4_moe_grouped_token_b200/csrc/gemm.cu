@@ -84,7 +84,7 @@ constexpr int kSlabRows = 32;
 // pieces in flight per warp.
 constexpr uint32_t kReqPiece = 5632;
 
-template <int BN_, int STAGES_, int ACC_, bool SWIGLU_>
+template <int BN_, int STAGES_, int ACC_, bool SWIGLU_, bool FUSED_ = false>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr int STAGES = STAGES_;
@@ -93,6 +93,8 @@ struct Cfg {
   // store / FP32 reduction (down); compiling only one keeps the other's
   // registers out of the kernel
   static constexpr bool SWIGLU = SWIGLU_;
+  // with the requantization of h fused into the launch (opt-in)
+  static constexpr bool FUSED = FUSED_;
   static constexpr int kABytes = BM * BK / 2;        // 16 KB of E2M1 codes
   static constexpr int kBBytes = BN * BK / 2;
   static constexpr int kSfaBytes = BM * BK / 16;     // four 512-byte atoms
@@ -123,6 +125,7 @@ struct Cfg {
 };
 
 using CfgGateUp = Cfg<256, 3, 1, true>;
+using CfgGateUpFused = Cfg<256, 3, 1, true, true>;
 using CfgDown = Cfg<256, 3, 1, false>;
 
 struct __align__(64) KParams {
@@ -373,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   const GemmArgs &a = P.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // requantize h inside this launch (SwiGLU epilogue, per-row amax)
-  const bool fused_requant = C::SWIGLU && a.req_q != nullptr && a.amax_h != nullptr &&
+  const bool fused_requant = C::FUSED && a.req_q != nullptr && a.amax_h != nullptr &&
                              a.amax_h_rows != 0;
 
   if (threadIdx.x == 0) {
@@ -908,7 +911,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
   // staging boxes; with plain 16-byte global stores of h instead, gate_up
   // measured 287 us against 266 us (the stage gains ~18 us, the stores lose
   // ~39 us), so the staged 3-stage ring stays.
-  if (a.epilogue == kEpiSwiGLU) return launch_cfg<CfgGateUp>(a, s);
+  if (a.epilogue == kEpiSwiGLU) {
+    const bool fused = a.req_q != nullptr && a.amax_h != nullptr && a.amax_h_rows != 0;
+    return fused ? launch_cfg<CfgGateUpFused>(a, s) : launch_cfg<CfgGateUp>(a, s);
+  }
   return launch_cfg<CfgDown>(a, s);
 }
 
