@@ -664,11 +664,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       // rows of this warp's 32-row slab all belong to the group?
       const bool slab_full = (row0 - g_pad) + quad * 32 + 32 <= g_cnt;
       if constexpr (C::SWIGLU) {
-        uint32_t hp[2][16];
         float m = 0.0f;
+        // h rows live at padded positions: the whole slab is stored (rows past
+        // the group's end are padding that nothing reads); each 32-column
+        // chunk is stored as soon as it is computed, which keeps the
+        // epilogue's registers within its share
         auto swiglu = [&](auto silu) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
+            uint32_t hp[16];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               float hh[2];
@@ -678,9 +682,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
                 const float u = __fmul_rn(__uint_as_float(v[(c + 2) % C::kChunks][i + q]), scale);
                 hh[q] = silu(g, u);
               }
-              hp[c][i / 2] = pack_bf16x2(hh[0], hh[1]);
-              m = fmax_abs_bf16(m, hp[c][i / 2]);
+              hp[i / 2] = pack_bf16x2(hh[0], hh[1]);
+              m = fmax_abs_bf16(m, hp[i / 2]);
             }
+            store_box(hp, (int32_t)(nt * 128 + half * 64 + c * 32), (int32_t)(row0 + quad * 32));
           }
         };
         // the fast SwiGLU form unless some gate value of the warp's tile
@@ -694,11 +699,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
           swiglu([](float g, float u) { return silu_mul(g, u); });
         else
           swiglu([](float g, float u) { return silu_mul_fast(g, u); });
-        // h rows live at padded positions: the whole slab is stored (rows past
-        // the group's end are padding that nothing reads)
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          store_box(hp[c], (int32_t)(nt * 128 + half * 64 + c * 32), (int32_t)(row0 + quad * 32));
         if (a.amax_h != nullptr) {
           if (a.amax_h_rows) {
             if (!fused_requant) {
