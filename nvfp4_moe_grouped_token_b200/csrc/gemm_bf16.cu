@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
               // (then 1 + e^g and 1 - s are 1 in binary32)
               const bool far = g < -64.0f;
               const float t = expf(g >= 0.0f ? -g : (far ? g + 64.0f : g));
-              const float sp = g >= 0.0f ? 1.0f / (1.0f + t) : (far ? t : t / (1.0f + t));
+              const float sp = (g >= 0.0f ? 1.0f : t) / (far ? 1.0f : 1.0f + t);   // one division
               const float sc = far ? kExpM64 : 1.0f;
               const float oms = far ? 1.0f : 1.0f - sp;
               const float gs = g * sp;
