@@ -609,6 +609,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       }
       ++chunk_id;
     };
+    // the plain store's 32-row x 64-column box (128-byte rows, 128-byte
+    // swizzle: chunk q of row r at q ^ (r & 7)), one 4 KB buffer per warp:
+    // half the TMA store requests of two 32 x 32 boxes
+    auto store_box64 = [&](const uint32_t (&w32)[32], int32_t x, int32_t y) {
+      if (lane == 0) bulk_wait_group_read<0>();   // the buffer's previous store has read it
+      __syncwarp();
+      const uint32_t base = stg_addr + (uint32_t)lane * 128;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st_shared_v4(base + (((uint32_t)q ^ ((uint32_t)lane & 7u)) << 4), w32[4 * q], w32[4 * q + 1], w32[4 * q + 2],
+                     w32[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&P.tmap_out, stg, x, y);
+        bulk_commit_group();
+      }
+    };
     // fused requantization: the warp's |h| maxima of a row are kept across
     // the n-tiles of an m-tile and folded into the row amax at its last
     // n-tile.  One tile later (its older bulk groups are then complete) lane
@@ -745,20 +763,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
         if (a.out_bf16 != nullptr) {
           const int64_t slab_row = a.out_padded ? row0 + quad * 32 : g_off + (row0 - g_pad) + quad * 32;
 #pragma unroll
-          for (int c = 0; c < C::kChunks; ++c) {
-            uint32_t w16[16];
+          for (int cc = 0; cc < C::kChunks / 2; ++cc) {
+            uint32_t w32[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w16[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[c][2 * i]), scale),
-                                   __fmul_rn(__uint_as_float(v[c][2 * i + 1]), scale));
+            for (int i = 0; i < 32; ++i) {
+              const int c = 2 * cc + (i >> 4), j = 2 * (i & 15);
+              w32[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[c][j]), scale),
+                                   __fmul_rn(__uint_as_float(v[c][j + 1]), scale));
+            }
             if (slab_full) {
-              store_box(w16, (int32_t)(col0 + c * 32), (int32_t)slab_row);
+              store_box64(w32, (int32_t)(col0 + cc * 64), (int32_t)slab_row);
             } else if (valid) {
               uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_bf16) +
-                                                     orow * a.N + col0 + c * 32);
+                                                     orow * a.N + col0 + cc * 64);
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_uint4(w32[4 * q], w32[4 * q + 1], w32[4 * q + 2], w32[4 * q + 3]);
             }
           }
         }
@@ -885,8 +905,10 @@ cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
   if (a.out_bf16 != nullptr) {
     // D: [rows][N] (compact rows never exceed rows_cap); h: [rows_cap][N/2]
     const uint64_t cols = a.epilogue == kEpiSwiGLU ? (uint64_t)(a.N / 2) : (uint64_t)a.N;
-    if (!encode_2d(&P.tmap_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out_bf16, cols,
-                   (uint64_t)a.rows_cap, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    // h: 32 x 32 boxes, 64-byte swizzle; D: 32 rows x 64 columns, 128-byte swizzle
+    const bool wide = a.epilogue != kEpiSwiGLU;
+    if (!encode_2d(&P.tmap_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out_bf16, cols, (uint64_t)a.rows_cap,
+                   wide ? 64 : 32, 32, wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
   const int64_t max_tiles = (a.rows_cap / BM) * (a.N / C::BN);
