@@ -339,6 +339,24 @@ int moe_expert_layer_from_logits(const void *x, const float *logits,
                                  size_t workspace_bytes,
                                  nvfp4moe_stream_t stream);
 
+/* The dense router in front of the routing: logits = x W_r^T in FP32, with
+ * BF16 operands on the tcgen05 tensor cores (kind::f16, FP32 accumulation).
+ * The pages list fusion and device-side metadata for the token path
+ * (www.aib.vote "miniTE report, NVFP4 RL stability", paragraph 4) and run
+ * Qwen3-30B-A3B, whose MoE router is this product; moe_route_permute or
+ * moe_expert_layer_from_logits take its output.
+ *   x          [T][H] BF16;  w_router [E][H] BF16 (device, 16-byte aligned)
+ *   logits     [T][E] FP32 (out)
+ *   workspace  moe_router_logits_workspace_size() bytes (device): the error
+ *              word at 0 (nvfp4moe_device_status), the GEMM's metadata
+ * Requirements: H % 64 == 0, E % 32 == 0, 1 <= E <= 1024, T < 2^30.
+ * Errors: NVFP4MOE_ERR_INVALID_ARG / _UNSUPPORTED_SHAPE / _MISALIGNED /
+ * _WORKSPACE before any launch; a CUDA error as NVFP4MOE_ERR_CUDA. */
+size_t moe_router_logits_workspace_size(void);
+int moe_router_logits(const void *x, const void *w_router, int64_t T, int64_t H,
+                      int E, float *logits, void *workspace,
+                      size_t workspace_bytes, nvfp4moe_stream_t stream);
+
 /* moe_expert_layer that also records CUDA events at its stage boundaries, so
  * a caller can time each kernel on the stream it runs on.  stage_events
  * (host array of 7 cudaEvent_t, entries may be NULL): [0] before the first

@@ -1075,4 +1075,50 @@ int moe_expert_layer_w4a8(const void *x, const int32_t *topk_idx, const float *t
                     stream, true);
 }
 
+// ------------------------------------------------------------ router GEMM --
+
+size_t moe_router_logits_workspace_size(void) { return 256; }
+
+int moe_router_logits(const void *x, const void *w_router, int64_t T, int64_t H, int E, float *logits,
+                      void *workspace, size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (T < 0 || H <= 0 || E < 1) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || E % 32 != 0 || H % 64 != 0 || T > (int64_t)1 << 30) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return NVFP4MOE_OK;
+  if (x == nullptr || w_router == nullptr || logits == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(workspace))
+    return NVFP4MOE_ERR_MISALIGNED;
+  if (workspace == nullptr || workspace_bytes < 256) return NVFP4MOE_ERR_WORKSPACE;
+  cudaStream_t s = st(stream);
+  // workspace: the error word at 0 (as in every workspace), the GEMM's group metadata at 64
+  int *err = static_cast<int *>(workspace);
+  int32_t *meta = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + 64);
+  const int64_t t_pad = (T + 127) / 128 * 128;
+  NVFP4MOE_TRY(cudaMemsetAsync(workspace, 0, 256, s));
+  NVFP4MOE_TRY(launch_router_meta(meta, T, t_pad, s));
+  // logits = x W_r^T: one group of T rows (A = x), B = W_r K-major; tile rows
+  // past T and past E read as zeros (the tensor maps hold the true row
+  // counts), and only the first E columns are stored, with leading dimension E
+  Bf16GemmArgs g;
+  g.mode = kBfRows;
+  g.a = x;
+  g.b = w_router;
+  g.b_mn = 0;
+  g.offsets = meta;
+  g.padded_offsets = meta + 2;
+  g.E = 1;
+  g.rows_cap = t_pad;
+  g.N = (E + 255) / 256 * 256;
+  g.K = H;
+  g.epilogue = kBfStore;
+  g.out_f32 = logits;
+  g.out_padded = 0;
+  g.a_rows = T;
+  g.b_rows = E;
+  g.n_store = E;
+  g.out_ld = E;
+  g.err = err;
+  NVFP4MOE_TRY(launch_bf16_gemm(g, s));
+  return NVFP4MOE_OK;
+}
+
 }  // extern "C"

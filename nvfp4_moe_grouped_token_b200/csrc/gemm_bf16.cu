@@ -363,8 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
                 dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
             }
           }
-          if (a.out_f32 != nullptr && valid) {
-            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + orow * a.N + col0 + c * 32);
+          const int64_t n_store = a.n_store ? a.n_store : a.N;
+          if (a.out_f32 != nullptr && valid && col0 + c * 32 < n_store) {
+            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + orow * (a.out_ld ? a.out_ld : a.N) + col0 + c * 32);
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               dst[i / 4] = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
@@ -970,13 +971,13 @@ cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
   int64_t tiles;
   if (a.mode == kBfRows) {
     if (a.K % BK != 0) return cudaErrorInvalidValue;
-    if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.K, (uint64_t)a.rows_cap, BK, BM, SW))
+    if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.K, (uint64_t)(a.a_rows ? a.a_rows : a.rows_cap), BK, BM, SW))
       return cudaErrorInvalidValue;
     if (a.b_mn) {
       if (!encode_2d_map(&P.tmap_b, BF, 2, a.b, (uint64_t)a.N, (uint64_t)(a.E * a.K), 64, BK, SW))
         return cudaErrorInvalidValue;
     } else {
-      if (!encode_2d_map(&P.tmap_b, BF, 2, a.b, (uint64_t)a.K, (uint64_t)(a.E * a.N), BK, BN, SW))
+      if (!encode_2d_map(&P.tmap_b, BF, 2, a.b, (uint64_t)a.K, (uint64_t)(a.b_rows ? a.b_rows : a.E * a.N), BK, BN, SW))
         return cudaErrorInvalidValue;
     }
     tiles = (a.rows_cap / BM) * (a.N / BN);

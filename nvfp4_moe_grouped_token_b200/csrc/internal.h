@@ -165,6 +165,10 @@ struct Bf16GemmArgs {
   // the per-expert decode scale applied to the accumulator in the epilogue
   const uint8_t *b_sf = nullptr;
   const float *s_dec_w = nullptr;
+  // kBfRows, K-major B (optional): the rows the A and B tensors really hold
+  // (tile rows past them read as zeros), and the FP32 output's valid columns
+  // and leading dimension (0: rows_cap, E * N, N and N)
+  int64_t a_rows = 0, b_rows = 0, n_store = 0, out_ld = 0;
   // kBfSwiGLUFwd: h is MXFP8 quantize-dequantized (W4A8); h_pre (optional)
   // receives the BF16 h before that, [rows_cap][I]
   int mxfp8_h = 0;
@@ -172,6 +176,8 @@ struct Bf16GemmArgs {
   int *err = nullptr;
 };
 cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s);
+// offsets {0, T} and padded offsets {0, Tpad} of the router GEMM's single group, in meta[0..3]
+cudaError_t launch_router_meta(int32_t *meta, int64_t T, int64_t Tpad, cudaStream_t s);
 
 // Backward helpers: gather x and dy rows into the padded grouped layout
 // (zeros on padding rows), the row weights, and ones for the dx combine

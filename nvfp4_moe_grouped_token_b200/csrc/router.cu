@@ -51,6 +51,25 @@ bool aligned16_ptr(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u
 }  // namespace
 }  // namespace nvfp4moe
 
+namespace nvfp4moe {
+namespace {
+// The one-group metadata of the router GEMM: offsets {0, T}, padded {0, Tpad}.
+__global__ void k_router_meta(int32_t *meta, int32_t T, int32_t Tpad) {
+  if (threadIdx.x == 0) {
+    meta[0] = 0;
+    meta[1] = T;
+    meta[2] = 0;
+    meta[3] = Tpad;
+  }
+}
+}  // namespace
+
+cudaError_t launch_router_meta(int32_t *meta, int64_t T, int64_t Tpad, cudaStream_t s) {
+  k_router_meta<<<1, 32, 0, s>>>(meta, (int32_t)T, (int32_t)Tpad);
+  return cudaGetLastError();
+}
+}  // namespace nvfp4moe
+
 using namespace nvfp4moe;
 
 extern "C" int moe_route_topk(const float *logits, int64_t T, int E, int k, int32_t *topk_idx, float *topk_w,

@@ -89,6 +89,8 @@ _SIGS = {
     "moe_expert_layer_w4a8": (_i32, [_vp, _vp, _vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights),
                                      _i64, _i64, _i64, _i32, _i32, _vp, _u32, _vp, _sz, _vp]),
     "nvfp4moe_last_cuda_error": (_i32, [ctypes.c_char_p, _sz]),
+    "moe_router_logits_workspace_size": (_sz, []),
+    "moe_router_logits": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _sz, _vp]),
     "nvfp4moe_num_sms": (_i32, []),
 }
 
@@ -187,6 +189,20 @@ def moe_route_topk(logits, k, topk_idx, topk_w, stream=None):
     T, E = logits.shape
     _check(lib().moe_route_topk(_p(logits), T, E, k, _p(topk_idx), _p(topk_w), _stream(stream)),
            "moe_route_topk")
+
+
+def moe_router_logits(x, w_router, logits, workspace=None, stream=None):
+    """moe_router_logits: logits [T][E] (FP32, out) = x [T][H] BF16 times
+    w_router [E][H] BF16, transposed."""
+    if workspace is None:
+        workspace = torch.empty(int(lib().moe_router_logits_workspace_size()), dtype=torch.uint8, device=x.device)
+    _dev(x, w_router, logits, workspace)
+    T, H = x.shape
+    E = w_router.shape[0]
+    _check(lib().moe_router_logits(_p(x), _p(w_router), T, H, E, _p(logits), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "moe_router_logits")
+    return workspace
 
 
 def moe_route_permute(logits, k, topk_idx, topk_w, offsets, padded_offsets, perm, inv_perm, workspace,

@@ -157,3 +157,54 @@ def test_layer_from_logits_equals_layer_with_routed_inputs():
         ops.moe_expert_layer(x, idx2, w2, wgu, wdn, y2, ws, flags)
         assert ops.device_status(ws) == 0
         assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), flags
+
+
+# ------------------------------------------------------------ router GEMM --
+
+def _router_inputs(T, H, E, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    w = (torch.randn(E, H, generator=g) * 0.02).to(torch.bfloat16)
+    return x, w
+
+
+@pytest.mark.parametrize("T,H,E", [(300, 256, 32), (129, 512, 128), (1000, 2048, 288), (64, 64, 1024)])
+def test_router_logits_match_oracle(T, H, E):
+    """logits = x W_r^T on the tensor cores against the oracle's exactly
+    rounded fp64 product, within 1e-5 * sum|x w| + 1e-6 (FP32 output).
+    Ragged T (tile rows past T read as zeros), E above 256 (a partial second
+    tile of weight rows) and H down to one K-step."""
+    x, w = _router_inputs(T, H, E, seed=T + E)
+    logits = torch.full((T, E), float("nan"), dtype=torch.float32, device="cuda")
+    ws = ops.moe_router_logits(x.cuda(), w.cuda(), logits)
+    assert ops.device_status(ws) == 0
+    ex, sa = cpp.gemm_rows(x.float().numpy().astype(np.float64), w.float().numpy().astype(np.float64), with_abs=True)
+    got = logits.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ex) <= 1e-5 * sa + 1e-6), float(np.max(np.abs(got - ex) / (1e-5 * sa + 1e-6)))
+
+
+def test_router_logits_moe30b_shape_then_routing():
+    """The Qwen3-30B-A3B router (T = 16384, H = 2048, E = 128), sampled rows
+    checked against the oracle; then routing from the GPU's logits matches
+    the oracle's router on the same logits (ids exact)."""
+    T, H, E, k = 16384, 2048, 128, 8
+    x, w = _router_inputs(T, H, E, seed=3)
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    ws = ops.moe_router_logits(x.cuda(), w.cuda(), logits)
+    assert ops.device_status(ws) == 0
+    rows = np.arange(7, T, 509)
+    ex, sa = cpp.gemm_rows(x[rows].float().numpy().astype(np.float64), w.float().numpy().astype(np.float64),
+                           with_abs=True)
+    got = logits.cpu().numpy()
+    assert np.all(np.abs(got[rows] - ex) <= 1e-5 * sa + 1e-6)
+    idx, wt = _route_gpu(logits.cpu(), k)
+    ref_idx, ref_w = cpp.route_topk(got, k)
+    assert np.array_equal(idx, ref_idx)
+    assert np.allclose(wt, ref_w, rtol=W_RTOL, atol=0)
+
+
+def test_router_logits_rejects_bad_shapes():
+    x, w = _router_inputs(16, 64, 48, seed=1)
+    logits = torch.empty(16, 48, dtype=torch.float32, device="cuda")
+    with pytest.raises(ops.NVFP4Error):        # E % 32 != 0
+        ops.moe_router_logits(x.cuda(), w.cuda(), logits)
