@@ -487,6 +487,35 @@ def measure_variant(cfg, dev, steps, warmup, kind):
                     "kind::f16 tensor cores; the whole step (routing, gather, both GEMMs, combine) is timed"}
 
 
+def measure_router(cfg, dev, steps, warmup):
+    """Time the dense router GEMM (moe_router_logits: logits = x W_r^T, BF16
+    operands, FP32 out) on the workload's shapes, W_r ~ N(0, 0.02)."""
+    from nvfp4_moe_grouped_token_b200 import ops
+
+    g = torch.Generator().manual_seed(91)
+    x = torch.randn(cfg.T, cfg.H, generator=g).to(torch.bfloat16).to(dev)
+    w = (torch.randn(cfg.E, cfg.H, generator=g) * 0.02).to(torch.bfloat16).to(dev)
+    logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        ops.moe_router_logits(x, w, logits, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        ops.moe_router_logits(x, w, logits, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    assert ops.device_status(ws) == 0
+    ms = e0.elapsed_time(e1) / steps
+    fl = 2.0 * cfg.T * cfg.H * cfg.E
+    byt = cfg.T * cfg.H * 2 + cfg.E * cfg.H * 2 + cfg.T * cfg.E * 4
+    pk = peaks()
+    return {"us": ms * 1e3, "tflops": fl / (ms * 1e-3) / 1e12, "gbs": byt / (ms * 1e-3) / 1e9,
+            "frac_hbm": byt / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "bound": "hbm",
+            "note": "x read once (67 MB for moe30b): HBM-bound at E = 128; tcgen05 kind::f16"}
+
+
 WORKLOAD_NAMES = {
     "toy": "toy NVFP4 MoE layer (E=4, T=256, top-2, K=256 -> N=512)",
     "dense4b": "dense Qwen3-4B-shaped W4A4 MLP (T=8192, 2560 -> 2x9728 -> 2560, 0.1% outlier channels x30)",
@@ -551,6 +580,7 @@ def run_ours(args, rank, world, local_rank):
         result["backward"] = measure_backward(cfg, dev, max(5, args.steps // 5), 2)
         torch.cuda.empty_cache()
     if world == 1 and not args.no_variants:
+        result["router_gemm"] = measure_router(cfg, dev, 20, 3)
         for kind in ("w4a16", "w4a8"):
             result[kind] = measure_variant(cfg, dev, max(5, args.steps // 5), 3, kind)
             torch.cuda.empty_cache()
