@@ -495,6 +495,74 @@ int moe_expert_layer_w4a8(const void *x, const int32_t *topk_idx,
                           uint32_t flags, void *workspace,
                           size_t workspace_bytes, nvfp4moe_stream_t stream);
 
+/* ------------------------------------------------- expert parallelism -- */
+/* The expert-parallel layer over G ranks, each owning El = E / G consecutive
+ * experts (expert e on rank e / El).  The library provides the steps around
+ * the two all-to-all exchanges, which the caller runs (NCCL over NVLink): the
+ * forward layer's data movement when its rows cross GPUs, in NVFP4 (4.5x
+ * fewer bytes than BF16).  Per-token scaling; results equal those of
+ * moe_expert_layer with NVFP4MOE_STRICT, bit for bit, whatever G.
+ *   1. source:  moe_ep_dispatch_pack: routing metadata and each token quantized
+ *      once into its k rows in compact sorted order (expert, token, slot), so
+ *      the rows for rank g are rows [offsets[g El], offsets[(g+1) El]).
+ *   2. exchange the [G][El] row counts and the rows (codes, row-major scales,
+ *      row S_dec), source-major on the receiver.
+ *   3. destination: moe_ep_arrange, moe_ep_experts, moe_ep_return.
+ *   4. exchange the D rows back (reverse splits); the source's concatenated
+ *      returns are its compact sorted D rows: moe_combine with its inv_perm.
+ * All pointers are device pointers, all buffers caller-allocated, all calls
+ * stream-ordered; errors as for moe_expert_layer; device-side checks go to
+ * each workspace's error word (nvfp4moe_device_status). */
+size_t moe_ep_dispatch_workspace_size(int64_t T, int E, int k);
+/*   x [T][H] BF16, topk_idx [T][k] (global expert ids)
+ *   q_send [T*k][H/2], sf_send [T*k][H/16] (UE4M3, row-major), sdec_send
+ *   [T*k] (FP32 per row), offsets [E+1] (compact, device), inv_perm [T][k]:
+ *   all written.  H % 256 == 0, 1 <= E <= 1024, 1 <= k <= 32. */
+int moe_ep_dispatch_pack(const void *x, const int32_t *topk_idx, int64_t T,
+                         int64_t H, int E, int k, uint8_t *q_send,
+                         uint8_t *sf_send, float *sdec_send, int32_t *offsets,
+                         int32_t *inv_perm, void *workspace,
+                         size_t workspace_bytes, nvfp4moe_stream_t stream);
+/* Rows of the padded grouped layout needed for rows_recv received rows over
+ * El local experts (each group padded to 128 rows). */
+int64_t moe_ep_rows_cap(int64_t rows_recv, int El);
+size_t moe_ep_arrange_workspace_size(int G, int El);
+/*   q_recv, sf_recv, sdec_recv  the received rows, source-major, each
+ *                source's rows in its (local expert, token, slot) order
+ *   counts       [G][El] int32 (device): rows received from source s for
+ *                local expert e
+ *   q_a, sf_a, sdec_a  the padded grouped layout (out): q_a [rows_cap][H/2],
+ *                sf_a K-step-major [H/256][rows_cap][16], sdec_a [rows_cap];
+ *                padding rows are zero
+ *   offsets, padded_offsets  [El+1] local groups (out)
+ *   workspace    moe_ep_arrange_workspace_size(G, El) bytes; keep it for
+ *                moe_ep_return (it holds the (source, expert) tables)
+ * Requirements: G * El <= 1024, H % 256 == 0, rows_cap >= moe_ep_rows_cap()
+ * and a multiple of 128. */
+int moe_ep_arrange(const uint8_t *q_recv, const uint8_t *sf_recv,
+                   const float *sdec_recv, const int32_t *counts, int G,
+                   int El, int64_t rows_recv, int64_t H, int64_t rows_cap,
+                   uint8_t *q_a, uint8_t *sf_a, float *sdec_a,
+                   int32_t *offsets, int32_t *padded_offsets, void *workspace,
+                   size_t workspace_bytes, nvfp4moe_stream_t stream);
+size_t moe_ep_experts_workspace_size(int64_t rows_cap, int64_t H, int64_t I);
+/* The local experts on the arranged rows: gate_up + SwiGLU, per-row NVFP4
+ * requantization of h, down.  w_gate_up / w_down hold the El local experts
+ * (prepared as for moe_expert_layer).  d [rows_recv][H] BF16 (out), compact
+ * local order (expert, then source, then the source's order). */
+int moe_ep_experts(const uint8_t *q_a, const uint8_t *sf_a,
+                   const float *sdec_a, const int32_t *offsets,
+                   const int32_t *padded_offsets, int El, int64_t rows_cap,
+                   const nvfp4moe_weights *w_gate_up,
+                   const nvfp4moe_weights *w_down, int64_t H, int64_t I,
+                   void *d, void *workspace, size_t workspace_bytes,
+                   nvfp4moe_stream_t stream);
+/* d_send [rows_recv][H] BF16 (out): the D rows in received order, ready for
+ * the reverse exchange.  workspace: the one moe_ep_arrange filled. */
+int moe_ep_return(const void *d, int G, int El, int64_t rows_recv, int64_t H,
+                  void *d_send, void *workspace, size_t workspace_bytes,
+                  nvfp4moe_stream_t stream);
+
 /* ---------------------------------------------------------- diagnostics -- */
 /* The hardware conversions the quantizer uses, exposed so their rounding can
  * be checked against the format definition: codes[i] = E2M1_rne_satfinite(y[i])

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libnvfp4moe.so")
 SOURCES = ["api.cu", "quantize.cu", "permute.cu", "gemm.cu", "gemm_bf16.cu", "backward.cu", "combine.cu", "probe.cu", "noalloc.cu",
-           "router.cu"]
+           "router.cu", "ep.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]

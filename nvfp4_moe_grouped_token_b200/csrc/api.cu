@@ -1121,4 +1121,254 @@ int moe_router_logits(const void *x, const void *w_router, int64_t T, int64_t H,
   return NVFP4MOE_OK;
 }
 
+// -------------------------------------------------- expert parallelism --
+
+size_t moe_ep_dispatch_workspace_size(int64_t T, int E, int k) {
+  if (T < 0 || E < 1 || k < 1) return 0;
+  Carve c;
+  c.take(kHeaderBytes);
+  c.take((E + 1) * 4);                      // padded offsets (the compact layout does not use them)
+  c.take(T * k * 4);                        // perm
+  c.take(permute_blocks(T) * E * 4);        // routing block counts
+  c.take(T * k * 4);                        // local ranks
+  return (size_t)c.off;
+}
+
+int moe_ep_dispatch_pack(const void *x, const int32_t *topk_idx, int64_t T, int64_t H, int E, int k, uint8_t *q_send,
+                         uint8_t *sf_send, float *sdec_send, int32_t *offsets, int32_t *inv_perm, void *workspace,
+                         size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (T < 0 || H <= 0 || E < 1 || k < 1 || k > 32) return NVFP4MOE_ERR_INVALID_ARG;
+  if (E > 1024 || H % 256 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (offsets == nullptr || workspace == nullptr) return NVFP4MOE_ERR_INVALID_ARG;
+  if (T > 0 && (x == nullptr || topk_idx == nullptr || q_send == nullptr || sf_send == nullptr ||
+                sdec_send == nullptr || inv_perm == nullptr))
+    return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q_send) || !aligned16(sf_send) || !aligned16(workspace))
+    return NVFP4MOE_ERR_MISALIGNED;
+  if (workspace_bytes < moe_ep_dispatch_workspace_size(T, E, k)) return NVFP4MOE_ERR_WORKSPACE;
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  Carve c;
+  int *err = reinterpret_cast<int *>(ws + c.take(kHeaderBytes));
+  int32_t *padded = reinterpret_cast<int32_t *>(ws + c.take((E + 1) * 4));
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + c.take(T * k * 4));
+  int32_t *block_counts = reinterpret_cast<int32_t *>(ws + c.take(permute_blocks(T) * E * 4));
+  int32_t *local_rank = reinterpret_cast<int32_t *>(ws + c.take(T * k * 4));
+  NVFP4MOE_TRY(cudaMemsetAsync(ws, 0, kHeaderBytes, s));
+  if (T == 0) {
+    NVFP4MOE_TRY(cudaMemsetAsync(offsets, 0, (E + 1) * 4, s));
+    return NVFP4MOE_OK;
+  }
+  PermuteParams pp;
+  pp.topk_idx = topk_idx;
+  pp.T = T;
+  pp.k = k;
+  pp.E = E;
+  pp.block_counts = block_counts;
+  pp.local_rank = local_rank;
+  pp.offsets = offsets;
+  pp.padded_offsets = padded;
+  pp.perm = perm;
+  pp.inv_perm = inv_perm;
+  pp.err = err;
+  pp.rows_cap = layer_rows_cap(T, k, E);
+  NVFP4MOE_TRY(launch_route_count(pp, s));
+  NVFP4MOE_TRY(launch_route_scan(pp, s));
+  // each token quantized once (per-token scale) and written to its k rows in
+  // compact sorted order: the destination offsets are the compact ones
+  QuantParams q;
+  q.x = x;
+  q.tasks = T;
+  q.K = H;
+  q.mode = kQuantScatter;
+  q.q = q_send;
+  q.sf = sf_send;
+  q.sf_layout = kSfRowMajor;
+  q.s_dec = sdec_send;
+  q.s_dec_rows = 1;
+  q.rows_cap = T * k;
+  q.topk_idx = topk_idx;
+  q.offsets = offsets;
+  q.padded_offsets = offsets;
+  q.k = k;
+  q.E = E;
+  q.local_rank = local_rank;
+  q.block_base = block_counts;
+  q.perm_out = perm;
+  q.inv_perm_out = inv_perm;
+  q.amax_rows = 1;
+  q.compute_row_amax = 1;
+  return cuda_rc(launch_quant(q, s));
+}
+
+int64_t moe_ep_rows_cap(int64_t rows_recv, int El) {
+  if (rows_recv < 0 || El < 1) return 0;
+  return layer_rows_cap(rows_recv, 1, El);
+}
+
+size_t moe_ep_arrange_workspace_size(int G, int El) {
+  if (G < 1 || El < 1) return 0;
+  return (size_t)(kHeaderBytes + round_up((int64_t)3 * G * El * 4, kAlign));
+}
+
+int moe_ep_arrange(const uint8_t *q_recv, const uint8_t *sf_recv, const float *sdec_recv, const int32_t *counts, int G,
+                   int El, int64_t rows_recv, int64_t H, int64_t rows_cap, uint8_t *q_a, uint8_t *sf_a, float *sdec_a,
+                   int32_t *offsets, int32_t *padded_offsets, void *workspace, size_t workspace_bytes,
+                   nvfp4moe_stream_t stream) {
+  if (G < 1 || El < 1 || rows_recv < 0 || H <= 0 || rows_cap < 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if ((int64_t)G * El > 1024 || H % 256 != 0 || rows_cap % 128 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows_cap < moe_ep_rows_cap(rows_recv, El)) return NVFP4MOE_ERR_WORKSPACE;
+  if (counts == nullptr || q_a == nullptr || sf_a == nullptr || sdec_a == nullptr || offsets == nullptr ||
+      padded_offsets == nullptr || workspace == nullptr ||
+      (rows_recv > 0 && (q_recv == nullptr || sf_recv == nullptr || sdec_recv == nullptr)))
+    return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(q_recv) || !aligned16(sf_recv) || !aligned16(q_a) || !aligned16(sf_a) || !aligned16(workspace))
+    return NVFP4MOE_ERR_MISALIGNED;
+  if (workspace_bytes < moe_ep_arrange_workspace_size(G, El)) return NVFP4MOE_ERR_WORKSPACE;
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int *err = reinterpret_cast<int *>(ws);
+  int32_t *tab = reinterpret_cast<int32_t *>(ws + kHeaderBytes);
+  NVFP4MOE_TRY(cudaMemsetAsync(ws, 0, kHeaderBytes, s));
+  NVFP4MOE_TRY(launch_ep_tables(counts, G, El, offsets, padded_offsets, tab, err, s));
+  EpArrangeParams a;
+  a.q_recv = q_recv;
+  a.sf_recv = sf_recv;
+  a.sdec_recv = sdec_recv;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.padded = padded_offsets;
+  a.tab = tab;
+  a.G = G;
+  a.El = El;
+  a.rows_recv = rows_recv;
+  a.H = H;
+  a.rows_cap = rows_cap;
+  a.q_a = q_a;
+  a.sf_a = sf_a;
+  a.sdec_a = sdec_a;
+  a.err = err;
+  NVFP4MOE_TRY(launch_ep_arrange(a, s));
+  return NVFP4MOE_OK;
+}
+
+int moe_ep_return(const void *d, int G, int El, int64_t rows_recv, int64_t H, void *d_send, void *workspace,
+                  size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (G < 1 || El < 1 || rows_recv < 0 || H <= 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if ((int64_t)G * El > 1024 || H % 8 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  if (workspace == nullptr || (rows_recv > 0 && (d == nullptr || d_send == nullptr))) return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(d) || !aligned16(d_send) || !aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  if (workspace_bytes < moe_ep_arrange_workspace_size(G, El)) return NVFP4MOE_ERR_WORKSPACE;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  return cuda_rc(launch_ep_return(d, reinterpret_cast<const int32_t *>(ws + kHeaderBytes), G * El, rows_recv, H,
+                                  d_send, reinterpret_cast<int *>(ws), st(stream)));
+}
+
+size_t moe_ep_experts_workspace_size(int64_t rows_cap, int64_t H, int64_t I) {
+  (void)H;
+  if (rows_cap < 0 || I <= 0) return 0;
+  Carve c;
+  c.take(kHeaderBytes);
+  c.take(rows_cap * I * 2);                 // h BF16
+  c.take(rows_cap * 4);                     // h row amax
+  c.take(rows_cap * I / 2);                 // h codes
+  c.take(rows_cap * I / 16);                // h scales (K-step-major)
+  c.take(rows_cap * 4);                     // h row S_dec
+  return (size_t)c.off;
+}
+
+int moe_ep_experts(const uint8_t *q_a, const uint8_t *sf_a, const float *sdec_a, const int32_t *offsets,
+                   const int32_t *padded_offsets, int El, int64_t rows_cap, const nvfp4moe_weights *w_gate_up,
+                   const nvfp4moe_weights *w_down, int64_t H, int64_t I, void *d, void *workspace,
+                   size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  if (El < 1 || rows_cap < 0 || H <= 0 || I <= 0) return NVFP4MOE_ERR_INVALID_ARG;
+  if (El > 1024 || H % 256 != 0 || I % 256 != 0 || rows_cap % 128 != 0) return NVFP4MOE_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_weights(w_gate_up, El, 2 * I, H);
+  if (rc != NVFP4MOE_OK) return rc;
+  if (!(w_gate_up->flags & NVFP4MOE_W_GATE_UP)) return NVFP4MOE_ERR_INVALID_ARG;
+  rc = check_weights(w_down, El, H, I);
+  if (rc != NVFP4MOE_OK) return rc;
+  if (q_a == nullptr || sf_a == nullptr || sdec_a == nullptr || offsets == nullptr || padded_offsets == nullptr ||
+      d == nullptr || workspace == nullptr)
+    return NVFP4MOE_ERR_INVALID_ARG;
+  if (!aligned16(q_a) || !aligned16(sf_a) || !aligned16(d) || !aligned16(workspace)) return NVFP4MOE_ERR_MISALIGNED;
+  if (workspace_bytes < moe_ep_experts_workspace_size(rows_cap, H, I)) return NVFP4MOE_ERR_WORKSPACE;
+  if (rows_cap == 0) return NVFP4MOE_OK;
+  cudaStream_t s = st(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  Carve c;
+  int *err = reinterpret_cast<int *>(ws + c.take(kHeaderBytes));
+  void *hb = ws + c.take(rows_cap * I * 2);
+  float *h_amax = reinterpret_cast<float *>(ws + c.take(rows_cap * 4));
+  uint8_t *hq = ws + c.take(rows_cap * I / 2);
+  uint8_t *hsf = ws + c.take(rows_cap * I / 16);
+  float *hsd = reinterpret_cast<float *>(ws + c.take(rows_cap * 4));
+  NVFP4MOE_TRY(cudaMemsetAsync(ws, 0, kHeaderBytes, s));
+  // padding rows keep amax 0: the requantization leaves them as zero codes
+  NVFP4MOE_TRY(cudaMemsetAsync(h_amax, 0, rows_cap * 4, s));
+  // gate_up grouped GEMM + SwiGLU epilogue (h in BF16, per-row amax of h)
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.q_a = q_a;
+  g.sf_a = sf_a;
+  g.s_dec_a = sdec_a;
+  g.s_dec_a_rows = 1;
+  g.q_w = w_gate_up->q;
+  g.sf_w = w_gate_up->sf;
+  g.s_dec_w = w_gate_up->s_dec;
+  g.offsets = offsets;
+  g.padded_offsets = padded_offsets;
+  g.E = El;
+  g.rows_cap = rows_cap;
+  g.N = 2 * I;
+  g.K = H;
+  g.epilogue = kEpiSwiGLU;
+  g.out_bf16 = hb;
+  g.out_padded = 1;
+  g.amax_h = h_amax;
+  g.amax_h_rows = 1;
+  g.err = err;
+  NVFP4MOE_TRY(launch_grouped_gemm(g, s));
+  // requantize h per row with the amax the epilogue reduced
+  QuantParams rq;
+  rq.x = hb;
+  rq.tasks = rows_cap;                      // the requantization walks the padded rows
+  rq.K = I;
+  rq.mode = kQuantRequant;
+  rq.amax_src = h_amax;
+  rq.amax_rows = 1;
+  rq.q = hq;
+  rq.sf = hsf;
+  rq.sf_layout = kSfKStep;
+  rq.s_dec = hsd;
+  rq.s_dec_rows = 1;
+  rq.rows_cap = rows_cap;
+  rq.offsets = offsets;
+  rq.padded_offsets = padded_offsets;
+  rq.E = El;
+  NVFP4MOE_TRY(launch_quant(rq, s));
+  // down grouped GEMM -> D (BF16, compact local rows)
+  GemmArgs dn;
+  std::memset(&dn, 0, sizeof(dn));
+  dn.q_a = hq;
+  dn.sf_a = hsf;
+  dn.s_dec_a = hsd;
+  dn.s_dec_a_rows = 1;
+  dn.q_w = w_down->q;
+  dn.sf_w = w_down->sf;
+  dn.s_dec_w = w_down->s_dec;
+  dn.offsets = offsets;
+  dn.padded_offsets = padded_offsets;
+  dn.E = El;
+  dn.rows_cap = rows_cap;
+  dn.N = H;
+  dn.K = I;
+  dn.epilogue = kEpiStore;
+  dn.out_bf16 = d;
+  dn.out_padded = 0;
+  dn.err = err;
+  NVFP4MOE_TRY(launch_grouped_gemm(dn, s));
+  return NVFP4MOE_OK;
+}
+
 }  // extern "C"

@@ -21,6 +21,7 @@ enum DeviceError : int {
   kDevBadExpert = 1,     // expert id out of range
   kDevDupExpert = 2,     // one token lists the same expert twice
   kDevTimeout = 3,       // a bounded wait ran out
+  kDevBadInput = 4,      // inconsistent counts or positions (expert-parallel exchange)
 };
 
 __device__ __forceinline__ void set_device_error(int *err, int code, int detail) {

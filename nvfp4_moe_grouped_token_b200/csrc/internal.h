@@ -176,6 +176,26 @@ struct Bf16GemmArgs {
   int *err = nullptr;
 };
 cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s);
+// Expert parallelism (ep.cu): tables from the [G][El] row counts, the
+// arrangement of received rows into the padded grouped layout, and the
+// return of D rows in received order.
+struct EpArrangeParams {
+  const uint8_t *q_recv = nullptr, *sf_recv = nullptr;   // [rows_recv][H/2], row-major [rows_recv][H/16]
+  const float *sdec_recv = nullptr;                       // [rows_recv]
+  const int32_t *counts = nullptr;                        // [G][El]
+  const int32_t *offsets = nullptr, *padded = nullptr;    // [El+1] (from the tables)
+  const int32_t *tab = nullptr;                           // recv_start, pad_start, cmp_start, [G*El] each
+  int G = 1, El = 1;
+  int64_t rows_recv = 0, H = 0, rows_cap = 0;
+  uint8_t *q_a = nullptr, *sf_a = nullptr;                // [rows_cap][H/2], K-step-major
+  float *sdec_a = nullptr;                                // [rows_cap]
+  int *err = nullptr;
+};
+cudaError_t launch_ep_tables(const int32_t *counts, int G, int El, int32_t *offsets, int32_t *padded, int32_t *tab,
+                             int *err, cudaStream_t s);
+cudaError_t launch_ep_arrange(const EpArrangeParams &a, cudaStream_t s);
+cudaError_t launch_ep_return(const void *d, const int32_t *tab, int P, int64_t rows_recv, int64_t H, void *d_send,
+                             int *err, cudaStream_t s);
 // offsets {0, T} and padded offsets {0, Tpad} of the router GEMM's single group, in meta[0..3]
 cudaError_t launch_router_meta(int32_t *meta, int64_t T, int64_t Tpad, cudaStream_t s);
 

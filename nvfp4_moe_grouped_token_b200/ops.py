@@ -90,6 +90,16 @@ _SIGS = {
                                      _i64, _i64, _i64, _i32, _i32, _vp, _u32, _vp, _sz, _vp]),
     "nvfp4moe_last_cuda_error": (_i32, [ctypes.c_char_p, _sz]),
     "moe_router_logits_workspace_size": (_sz, []),
+    "moe_ep_dispatch_workspace_size": (_sz, [_i64, _i32, _i32]),
+    "moe_ep_dispatch_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_ep_rows_cap": (_i64, [_i64, _i32]),
+    "moe_ep_arrange_workspace_size": (_sz, [_i32, _i32]),
+    "moe_ep_arrange": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                              _vp]),
+    "moe_ep_experts_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "moe_ep_experts": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights),
+                              _i64, _i64, _vp, _vp, _sz, _vp]),
+    "moe_ep_return": (_i32, [_vp, _i32, _i32, _i64, _i64, _vp, _vp, _sz, _vp]),
     "moe_router_logits": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _sz, _vp]),
     "nvfp4moe_num_sms": (_i32, []),
 }
@@ -205,6 +215,64 @@ def moe_router_logits(x, w_router, logits, workspace=None, stream=None):
     return workspace
 
 
+# ------------------------------------------------- expert parallelism --
+# Argument marshalling for the library's expert-parallel steps; the
+# orchestration around the exchanges is in nvfp4_moe_grouped_token_b200.ep.
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def moe_ep_dispatch_pack(x, topk_idx, E, q_send, sf_send, sdec_send, offsets, inv_perm, workspace, stream=None):
+    _dev(x, topk_idx, q_send, sf_send, sdec_send, offsets, inv_perm, workspace)
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    _check(lib().moe_ep_dispatch_pack(_p(x), _p(topk_idx), T, H, E, k, _p(q_send), _p(sf_send), _p(sdec_send),
+                                      _p(offsets), _p(inv_perm), _p(workspace), _nbytes(workspace), _stream(stream)),
+           "moe_ep_dispatch_pack")
+
+
+def moe_ep_dispatch_workspace_size(T, E, k) -> int:
+    return int(lib().moe_ep_dispatch_workspace_size(T, E, k))
+
+
+def moe_ep_rows_cap(rows_recv, El) -> int:
+    return int(lib().moe_ep_rows_cap(rows_recv, El))
+
+
+def moe_ep_arrange_workspace_size(G, El) -> int:
+    return int(lib().moe_ep_arrange_workspace_size(G, El))
+
+
+def moe_ep_arrange(q_recv, sf_recv, sdec_recv, counts, G, El, H, rows_cap, q_a, sf_a, sdec_a, offsets,
+                   padded_offsets, workspace, stream=None):
+    _dev(q_recv, sf_recv, sdec_recv, counts, q_a, sf_a, sdec_a, offsets, padded_offsets, workspace)
+    rows_recv = q_recv.shape[0]
+    _check(lib().moe_ep_arrange(_p(q_recv), _p(sf_recv), _p(sdec_recv), _p(counts), G, El, rows_recv, H, rows_cap,
+                                _p(q_a), _p(sf_a), _p(sdec_a), _p(offsets), _p(padded_offsets), _p(workspace),
+                                _nbytes(workspace), _stream(stream)), "moe_ep_arrange")
+
+
+def moe_ep_experts_workspace_size(rows_cap, H, I) -> int:
+    return int(lib().moe_ep_experts_workspace_size(rows_cap, H, I))
+
+
+def moe_ep_experts(q_a, sf_a, sdec_a, offsets, padded_offsets, rows_cap, w_gate_up: "NVFP4Weights",
+                   w_down: "NVFP4Weights", d, workspace, stream=None):
+    _dev(q_a, sf_a, sdec_a, offsets, padded_offsets, d, workspace)
+    gu, dn = w_gate_up.struct(), w_down.struct()
+    _check(lib().moe_ep_experts(_p(q_a), _p(sf_a), _p(sdec_a), _p(offsets), _p(padded_offsets), w_down.E, rows_cap,
+                                ctypes.byref(gu), ctypes.byref(dn), w_down.N, w_down.K, _p(d), _p(workspace),
+                                _nbytes(workspace), _stream(stream)), "moe_ep_experts")
+
+
+def moe_ep_return(d, G, El, d_send, workspace, stream=None):
+    _dev(d, d_send, workspace)
+    rows_recv, H = d_send.shape
+    _check(lib().moe_ep_return(_p(d), G, El, rows_recv, H, _p(d_send), _p(workspace), _nbytes(workspace),
+                               _stream(stream)), "moe_ep_return")
+
+
 def moe_route_permute(logits, k, topk_idx, topk_w, offsets, padded_offsets, perm, inv_perm, workspace,
                       stream=None):
     """moe_route_permute: router top-k fused with the routing histogram, then
@@ -264,6 +332,13 @@ class NVFP4Weights:
     def struct(self) -> _Weights:
         return _Weights(self.q.data_ptr(), self.sf.data_ptr(), self.s_dec.data_ptr(),
                         self.amax.data_ptr(), self.E, self.N, self.K, self.flags)
+
+    def experts(self, lo: int, hi: int) -> "NVFP4Weights":
+        """Experts [lo, hi) as views of the same buffers (each expert's codes,
+        scales and S_dec are its own)."""
+        per = self.N * self.K // 16
+        return NVFP4Weights(q=self.q[lo:hi], sf=self.sf[lo * per:hi * per], s_dec=self.s_dec[lo:hi],
+                            amax=self.amax[lo:hi], E=hi - lo, N=self.N, K=self.K, flags=self.flags)
 
 
 def nvfp4_prepare_weights(w: torch.Tensor, gate_up: bool, stream=None) -> NVFP4Weights:
