@@ -516,6 +516,51 @@ def measure_router(cfg, dev, steps, warmup):
             "note": "x read once (67 MB for moe30b): HBM-bound at E = 128; tcgen05 kind::f16"}
 
 
+def measure_ep(cfg, dev, steps, warmup, G):
+    """The expert-parallel pipeline (nvfp4_moe_grouped_token_b200.ep) with G
+    ranks driven by this process on one GPU: dispatch, exchanges as device
+    copies, arrange, experts, return, combine, including the one host read of
+    the offsets per rank that sizes the exchange.  Reports the step time and
+    the bytes that would cross NVLink per step (NVFP4 rows out, BF16 D back)."""
+    from nvfp4_moe_grouped_token_b200 import ep, ops
+
+    inp = workloads.layer_inputs(cfg)
+    wgu = ops.nvfp4_prepare_weights(inp["w_gate_up"].to(dev), gate_up=True)
+    wdn = ops.nvfp4_prepare_weights(inp["w_down"].to(dev), gate_up=False)
+    b = [cfg.T * g // G for g in range(G + 1)]
+    xs = [inp["x"][b[g]:b[g + 1]].contiguous().to(dev) for g in range(G)]
+    idxs = [inp["topk_idx"][b[g]:b[g + 1]].contiguous().to(dev) for g in range(G)]
+    tws = [inp["topk_w"][b[g]:b[g + 1]].contiguous().to(dev) for g in range(G)]
+    ys = [torch.empty(b[g + 1] - b[g], cfg.H, dtype=torch.bfloat16, device=dev) for g in range(G)]
+    wgus = [ep.local_weights(wgu, g, G) for g in range(G)]
+    wdns = [ep.local_weights(wdn, g, G) for g in range(G)]
+
+    def step():
+        return ep.moe_expert_layer_ep_local(xs, idxs, tws, wgus, wdns, ys, cfg.E)
+
+    for _ in range(warmup):
+        assert step() == 0
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    # rows that leave their rank: each routed row whose expert lives elsewhere
+    idx = inp["topk_idx"]
+    owner = idx // (cfg.E // G)
+    src = torch.repeat_interleave(torch.arange(G), torch.tensor([b[g + 1] - b[g] for g in range(G)]))
+    remote = int((owner != src[:, None]).sum())
+    row_out = cfg.H // 2 + cfg.H // 16 + 4
+    return {"simulated_ranks": G, "ms_per_step": ms, "tokens_per_s": cfg.T / (ms * 1e-3),
+            "remote_rows": remote, "nvlink_bytes_per_step": remote * (row_out + 2 * cfg.H),
+            "bf16_dispatch_bytes_would_be": remote * (2 * cfg.H + 2 * cfg.H),
+            "note": "one GPU drives all ranks (exchanges are device copies); results equal the strict layer "
+                    "bit for bit (tests/test_gpu_ep.py)"}
+
+
 WORKLOAD_NAMES = {
     "toy": "toy NVFP4 MoE layer (E=4, T=256, top-2, K=256 -> N=512)",
     "dense4b": "dense Qwen3-4B-shaped W4A4 MLP (T=8192, 2560 -> 2x9728 -> 2560, 0.1% outlier channels x30)",
@@ -581,6 +626,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
     if world == 1 and not args.no_variants:
         result["router_gemm"] = measure_router(cfg, dev, 20, 3)
+        result["expert_parallel"] = measure_ep(cfg, dev, 5, 2, 4)
+        torch.cuda.empty_cache()
         for kind in ("w4a16", "w4a8"):
             result[kind] = measure_variant(cfg, dev, max(5, args.steps // 5), 3, kind)
             torch.cuda.empty_cache()
