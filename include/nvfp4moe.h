@@ -499,7 +499,7 @@ int moe_expert_layer_w4a8(const void *x, const int32_t *topk_idx,
 /* The expert-parallel layer over G ranks, each owning El = E / G consecutive
  * experts (expert e on rank e / El).  The library provides the steps around
  * the two all-to-all exchanges, which the caller runs (NCCL over NVLink): the
- * forward layer's data movement when its rows cross GPUs, in NVFP4 (4.5x
+ * forward layer's data movement when its rows cross GPUs, in NVFP4 (3.6x
  * fewer bytes than BF16).  Per-token scaling; results equal those of
  * moe_expert_layer with NVFP4MOE_STRICT, bit for bit, whatever G.
  *   1. source:  moe_ep_dispatch_pack: routing metadata and each token quantized
