@@ -1009,6 +1009,7 @@ int w4ax_layer(const void *x, const int32_t *topk_idx, const float *topk_w, cons
   g1.out_bf16 = h;
   g1.out_padded = 1;
   g1.mxfp8_h = mxfp8 ? 1 : 0;
+  g1.w4_wide = 1;
   g1.h_pre = keep_h_pre ? ws + L.v[8] : nullptr;
   NVFP4MOE_TRY(launch_bf16_gemm(g1, s));
   // down with NVFP4 weights -> D (compact sorted rows)
@@ -1022,6 +1023,7 @@ int w4ax_layer(const void *x, const int32_t *topk_idx, const float *topk_w, cons
   g2.epilogue = kBfStore;
   g2.out_bf16 = d;
   g2.out_padded = 0;
+  g2.w4_wide = 1;
   NVFP4MOE_TRY(launch_bf16_gemm(g2, s));
   NVFP4MOE_TRY(launch_combine(d, inv_perm, topk_w, T, k, H, y, s));
   return NVFP4MOE_OK;

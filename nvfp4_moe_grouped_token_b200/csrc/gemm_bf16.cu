@@ -482,29 +482,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
 //   (m-tile = which half of the warps, TMEM lane quarter = warp % 4);
 //   warps 10-17: converters, one half row per lane and K-step.
 namespace w4 {
-constexpr int RS = 4;
-constexpr int CS = 2;
-constexpr int WN = 128;                                   // weight rows per unit
-constexpr int kA2Bytes = 2 * kABytes;                     // A of two m-tiles
-constexpr int kCodesBytes = WN * BK / 2;                  // 4 KB
-constexpr int kSfBytes = 2 * 512;                         // two scale atoms
-constexpr int kRawBytes = kA2Bytes + kCodesBytes + kSfBytes;
-constexpr int kConvBytes = WN * BK * 2;                   // 16 KB
-constexpr int kAccCols = 2 * WN;                          // one buffer: two m-tiles
 constexpr int kThreads = 576;
 constexpr int kEpiWarp0 = 2, kConvWarp0 = 10, kConvWarps = 8;
-constexpr size_t kConvOff = (size_t)RS * kRawBytes;
-constexpr size_t kStagingOff = kConvOff + (size_t)CS * kConvBytes;
-constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
-constexpr size_t kPairsOff = kBarrierOff + 256;           // + (E + 1) int32 pair prefix
-constexpr size_t kSmemMax = kPairsOff + 4 * 1025 + 1024;  // + up to 1023 bytes of alignment
-static_assert(kRawBytes % 1024 == 0 && kConvBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
-static_assert(kSmemMax <= 232448, "shared memory budget");
-static_assert(kConvWarps * 32 == 2 * WN, "each converter lane covers one half row");
-static_assert(ACC * kAccCols <= 512, "TMEM budget");
-// Instruction descriptor as idesc_bf16 with N = 128, both operands K-major.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(WN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+constexpr int CS = 2;
+
+// WN weight rows per unit: 128 (two accumulator buffers of 2 x 128 columns,
+// 4 raw stages) or 256 (one buffer of 2 x 256 columns, 3 raw stages; fewer
+// load rows and conversions per FLOP, the epilogue no longer overlapped).
+template <int WN_>
+struct Cfg {
+  static constexpr int WN = WN_;
+  static constexpr int RS = WN == 128 ? 4 : 3;
+  static constexpr int ACC = WN == 128 ? 2 : 1;
+  static constexpr int kA2Bytes = 2 * kABytes;             // A of two m-tiles
+  static constexpr int kCodesBytes = WN * BK / 2;          // two boxes of WN/2 rows x 32 bytes
+  static constexpr int kSfBytes = 2 * 512;                 // the two scale atoms holding those rows
+  static constexpr int kRawBytes = kA2Bytes + kCodesBytes + kSfBytes;
+  static constexpr int kConvBytes = WN * BK * 2;
+  static constexpr int kAccCols = 2 * WN;                  // one buffer: two m-tiles
+  static constexpr int kHalfRowsPerLane = WN / 128;        // converter: K-half rows per lane
+  static constexpr size_t kConvOff = (size_t)RS * kRawBytes;
+  static constexpr size_t kStagingOff = kConvOff + (size_t)CS * kConvBytes;
+  static constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
+  static constexpr size_t kPairsOff = kBarrierOff + 256;   // + (E + 1) int32 pair prefix
+  static constexpr size_t kSmemMax = kPairsOff + 4 * 1025 + 1024;   // + up to 1023 bytes of alignment
+  // Instruction descriptor as idesc_bf16 with N = WN, both operands K-major.
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(WN >> 3) << 17) |
+                                     ((uint32_t)(BM >> 4) << 24);
+  static_assert(WN == 128 || WN == 256, "unit width");
+  static_assert(kRawBytes % 1024 == 0 && kConvBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kSmemMax <= 232448, "shared memory budget");
+  static_assert(kConvWarps * 32 * kHalfRowsPerLane == 2 * WN, "converter lanes cover the half rows");
+  static_assert(ACC * kAccCols <= 512, "TMEM budget");
+  static_assert((3 * RS + 2 * CS + 2 * ACC + 1) * 8 + 12 <= 256, "barrier area");
+};
 
 // A unit's m-tiles and weight rows.
 struct Unit {
@@ -512,10 +523,11 @@ struct Unit {
   int64_t m0;       // first padded row of the first m-tile
   bool two;         // a second m-tile at m0 + 128
   int nt;           // weight-row tile
-  int64_t wrow0;    // first weight row of each 64-row half (global row of the [E*N] codes)
+  int64_t wrow0;    // first weight row of each WN/2-row half (global row of the [E*N] codes)
   int64_t wrow1;
 };
 
+template <int WN>
 __device__ __forceinline__ Unit unit_of(const Bf16GemmArgs &a, const int32_t *pairs, int64_t u, int n_tiles,
                                         int64_t rows_cap) {
   Unit r;
@@ -531,9 +543,15 @@ __device__ __forceinline__ Unit unit_of(const Bf16GemmArgs &a, const int32_t *pa
   const int64_t g_hi = min((int64_t)__ldg(a.padded_offsets + lo + 1), rows_cap);
   r.m0 = g_lo + 2 * BM * (p - pairs[lo]);
   r.two = r.m0 + BM < g_hi;
-  const bool gate_up = a.epilogue == kBfSwiGLUFwd;
-  r.wrow0 = (int64_t)r.e * a.N + (gate_up ? 256 * (r.nt >> 1) + 64 * (r.nt & 1) : (int64_t)WN * r.nt);
-  r.wrow1 = r.wrow0 + (gate_up ? 128 : 64);
+  if (a.epilogue == kBfSwiGLUFwd) {
+    // WN/2 gate rows of a 256-row block (128 gate, then 128 up) and the matching up rows
+    constexpr int per_block = 256 / WN;
+    r.wrow0 = (int64_t)r.e * a.N + 256 * (r.nt / per_block) + (WN / 2) * (r.nt % per_block);
+    r.wrow1 = r.wrow0 + 128;
+  } else {
+    r.wrow0 = (int64_t)r.e * a.N + (int64_t)WN * r.nt;
+    r.wrow1 = r.wrow0 + WN / 2;
+  }
   return r;
 }
 }  // namespace w4
@@ -595,12 +613,17 @@ __device__ __forceinline__ uint32_t ld_shared_u16(uint32_t saddr) {
   return v;
 }
 
+template <class C>
 __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_constant__ BParams P) {
   using namespace w4;
+  constexpr int WN = C::WN, RS = C::RS, ACC = C::ACC;
+  constexpr int kA2Bytes = C::kA2Bytes, kCodesBytes = C::kCodesBytes, kRawBytes = C::kRawBytes;
+  constexpr int kConvBytes = C::kConvBytes, kAccCols = C::kAccCols;
+  constexpr size_t kConvOff = C::kConvOff;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + w4::kBarrierOff);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff);
   uint64_t *empty = full + RS;
   uint64_t *cfull = empty + RS;
   uint64_t *cempty = cfull + CS;
@@ -610,7 +633,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *never = reinterpret_cast<int *>(tmem_slot + 2);
-  int32_t *pairs = reinterpret_cast<int32_t *>(smem + kPairsOff);   // [E + 1]
+  int32_t *pairs = reinterpret_cast<int32_t *>(smem + C::kPairsOff);   // [E + 1]
 
   const Bf16GemmArgs &a = P.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -679,7 +702,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
       uint32_t p = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
+        const Unit un = unit_of<WN>(a, pairs, t, n_tiles, a.rows_cap);
         const uint8_t *sf0 = a.b_sf + (un.wrow0 >> 7) * k_atoms * 512;
         const uint8_t *sf1 = a.b_sf + (un.wrow1 >> 7) * k_atoms * 512;
         const uint32_t bytes = un.two ? kRawBytes : kRawBytes - kABytes;
@@ -708,7 +731,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
       uint32_t p = 0, it = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
+        const Unit un = unit_of<WN>(a, pairs, t, n_tiles, a.rows_cap);
         const uint32_t as = it % ACC;
         const uint32_t acc = tmem + as * kAccCols;
         if (!mbar_wait_bounded(&acc_empty[as], ((it / ACC) & 1u) ^ 1u, abort_flag, a.err, 540)) break;
@@ -726,8 +749,8 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t accum = (kt | kk) != 0 ? 1u : 0u;
-            mma_bf16(acc, dk | (a16 + kk * 2), dk | (b16 + kk * 2), kIdesc, accum);
-            if (un.two) mma_bf16(acc + WN, dk | (a16 + kABytes / 16 + kk * 2), dk | (b16 + kk * 2), kIdesc, accum);
+            mma_bf16(acc, dk | (a16 + kk * 2), dk | (b16 + kk * 2), C::kIdesc, accum);
+            if (un.two) mma_bf16(acc + WN, dk | (a16 + kABytes / 16 + kk * 2), dk | (b16 + kk * 2), C::kIdesc, accum);
           }
           tc_commit(&empty[st]);
           tc_commit(&cempty[cs]);
@@ -739,28 +762,37 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     }
   } else if (warp >= kConvWarp0) {
     // ------------------------------------------------------- converters
-    // Lane l of converter warp w covers K-half (l & 1) of B row
-    // r = 16w + l/2 (rows 0-63 from the first 64-row box, 64-127 from the
-    // second): its 16-byte code loads are contiguous across the warp, and its
-    // 16-byte stores land in distinct banks within every quarter warp under
-    // the 128-byte swizzle.
+    // Lane l of converter warp w covers K-half (l & 1) of the B rows
+    // r = 16 (kHalfRowsPerLane w + j) + l/2, j < kHalfRowsPerLane (rows below
+    // WN/2 from the first box, the rest from the second): its 16-byte code
+    // loads are contiguous across the warp, and its 16-byte stores land in
+    // distinct banks within every quarter warp under the 128-byte swizzle.
+    constexpr int HR = C::kHalfRowsPerLane;
     const int cw = warp - kConvWarp0;
     const int hk = lane & 1;
-    const int r = 16 * cw + (lane >> 1);
-    const int half_box = r >> 6;
     const uint32_t smem0 = smem_u32(smem);
-    const uint32_t code_off = (uint32_t)(kA2Bytes + r * 32 + hk * 16);
-    uint32_t dst_off[4];
+    int r[HR];
+    uint32_t code_off[HR], dst_off[HR][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst_off[i] = (uint32_t)(r * 128) + ((uint32_t)((4 * hk + i) ^ (r & 7)) << 4);
+    for (int j = 0; j < HR; ++j) {
+      r[j] = 16 * (HR * cw + j) + (lane >> 1);
+      code_off[j] = (uint32_t)(kA2Bytes + r[j] * 32 + hk * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst_off[j][i] = (uint32_t)(r[j] * 128) + ((uint32_t)((4 * hk + i) ^ (r[j] & 7)) << 4);
+    }
     uint32_t p = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
-      // the row's place in its 128-row scale atom
-      const int ra = (int)(((half_box ? un.wrow1 : un.wrow0) & 127) + (r & 63));
-      const uint32_t sf_off = (uint32_t)(kA2Bytes + kCodesBytes + half_box * 512 + (ra & 31) * 16 + (ra >> 5) * 4 +
-                                         2 * hk);
+      const Unit un = unit_of<WN>(a, pairs, t, n_tiles, a.rows_cap);
+      // each row's place in its 128-row scale atom
+      uint32_t sf_off[HR];
+#pragma unroll
+      for (int j = 0; j < HR; ++j) {
+        const int half_box = r[j] / (WN / 2);
+        const int ra = (int)(((half_box ? un.wrow1 : un.wrow0) & 127) + (r[j] % (WN / 2)));
+        sf_off[j] = (uint32_t)(kA2Bytes + kCodesBytes + half_box * 512 + (ra & 31) * 16 + (ra >> 5) * 4 + 2 * hk);
+      }
       for (int kt = 0; kt < ksteps; ++kt, ++p) {
         const uint32_t st = p % RS, cs = p % CS;
         if (!mbar_wait_bounded(&full[st], (p / RS) & 1u, abort_flag, a.err, 550) ||
@@ -770,18 +802,26 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
         }
         const uint32_t raw = smem0 + st * (uint32_t)kRawBytes;
         const uint32_t dst = smem0 + (uint32_t)kConvOff + cs * (uint32_t)kConvBytes;
-        const uint4 q = ld_shared_v4(raw + code_off);
-        const uint32_t sc = ld_shared_u16(raw + sf_off);
-        uint32_t s2[2];
-        ue4m3x2_to_bf16x2(sc, s2[0], s2[1]);
-        const uint32_t cw4[4] = {q.x, q.y, q.z, q.w};
+        uint4 q[HR];
+        uint32_t sc[HR];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t w[4];
-          e2m1x8_to_bf16x2(cw4[i], w);
+        for (int j = 0; j < HR; ++j) {
+          q[j] = ld_shared_v4(raw + code_off[j]);
+          sc[j] = ld_shared_u16(raw + sf_off[j]);
+        }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) w[u] = mul_bf16x2(w[u], s2[i >> 1]);
-          st_shared_v4(dst + dst_off[i], w[0], w[1], w[2], w[3]);
+        for (int j = 0; j < HR; ++j) {
+          uint32_t s2[2];
+          ue4m3x2_to_bf16x2(sc[j], s2[0], s2[1]);
+          const uint32_t cw4[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+            e2m1x8_to_bf16x2(cw4[i], w);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w[u] = mul_bf16x2(w[u], s2[i >> 1]);
+            st_shared_v4(dst + dst_off[j][i], w[0], w[1], w[2], w[3]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -794,7 +834,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     const int quad = warp & 3;
     const int half = ew >> 2;              // which m-tile of the unit
     const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-    uint8_t *stg = smem + w4::kStagingOff + (size_t)ew * kStagingPerWarp;
+    uint8_t *stg = smem + C::kStagingOff + (size_t)ew * kStagingPerWarp;
     const uint32_t stg_addr = smem_u32(stg);
     uint32_t chunk_id = 0, it = 0;
     auto store_box = [&](const uint32_t (&w16)[16], int32_t x, int32_t y) {
@@ -817,7 +857,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
     };
     const int64_t rows_total = (int64_t)__ldg(a.offsets + a.E);
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const Unit un = unit_of(a, pairs, t, n_tiles, a.rows_cap);
+      const Unit un = unit_of<WN>(a, pairs, t, n_tiles, a.rows_cap);
       const uint32_t as = it % ACC;
       const float scale = __ldg(a.s_dec_w + un.e);
       if (!mbar_wait_bounded(&acc_full[as], (it / ACC) & 1u, abort_flag, a.err, 560)) break;
@@ -829,15 +869,15 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
       const uint32_t tacc = tlane + as * kAccCols + half * WN;
       const int64_t mrow0 = un.m0 + half * BM;
       if (a.epilogue == kBfSwiGLUFwd) {
-        // gate columns [0, 64), up columns [64, 128) of the unit; h columns
-        // 64 nt + [0, 64), every padded row of the slab
+        // gate columns [0, WN/2), up columns [WN/2, WN) of the unit; h
+        // columns (WN/2) nt + [0, WN/2), every padded row of the slab
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < WN / 64; ++c) {
           uint32_t vg[32], vu[32];
           tmem_ld_32cols(tacc + c * 32, vg);
-          tmem_ld_32cols(tacc + 64 + c * 32, vu);
+          tmem_ld_32cols(tacc + WN / 2 + c * 32, vu);
           tmem_ld_wait();
-          if (c == 1) release(as);
+          if (c == WN / 64 - 1) release(as);
           uint32_t w16[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -848,7 +888,7 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
                                __fmul_rn(__uint_as_float(vu[2 * i + q]), scale));
             w16[i] = pack_bf16x2(hh[0], hh[1]);
           }
-          const int32_t hcol = (int32_t)(64 * un.nt + c * 32);
+          const int32_t hcol = (int32_t)((WN / 2) * un.nt + c * 32);
           if (a.mxfp8_h) {
             // W4A8: the BF16 h of these 32 columns is one MXFP8 block
             if (a.h_pre != nullptr) {
@@ -880,11 +920,11 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
         const int64_t slab_row = a.out_padded ? mrow0 + quad * 32 : g_off + (mrow0 - g_pad) + quad * 32;
         const int64_t col0 = (int64_t)WN * un.nt;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < WN / 32; ++c) {
           uint32_t v[32];
           tmem_ld_32cols(tacc + c * 32, v);
           tmem_ld_wait();
-          if (c == 3) release(as);
+          if (c == WN / 32 - 1) release(as);
           uint32_t w16[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -915,17 +955,19 @@ __global__ void __launch_bounds__(w4::kThreads, 1) k_w4a16_gemm(const __grid_con
 
 }  // namespace
 
-static cudaError_t launch_w4a16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
+template <int WN>
+static cudaError_t launch_w4a16_cfg(const Bf16GemmArgs &a, cudaStream_t s) {
+  using C = w4::Cfg<WN>;
   if (a.mode != kBfRows || a.b_mn || a.s_dec_w == nullptr || a.out_bf16 == nullptr || a.K % BK != 0 ||
       a.E < 1 || a.E > 1024 || (a.epilogue != kBfStore && a.epilogue != kBfSwiGLUFwd) ||
-      (a.epilogue == kBfSwiGLUFwd && (!a.out_padded || a.N % 256 != 0)) || a.N % w4::WN != 0)
+      (a.epilogue == kBfSwiGLUFwd && (!a.out_padded || a.N % 256 != 0)) || a.N % WN != 0)
     return cudaErrorInvalidValue;
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (configured_device != dev) {
-    err = cudaFuncSetAttribute(k_w4a16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)w4::kSmemMax);
+    err = cudaFuncSetAttribute(k_w4a16_gemm<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemMax);
     if (err != cudaSuccess) return err;
     configured_device = dev;
   }
@@ -934,22 +976,26 @@ static cudaError_t launch_w4a16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!encode_2d_map(&P.tmap_a, BF, 2, a.a, (uint64_t)a.K, (uint64_t)a.rows_cap, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // weight codes: boxes of 64 rows x 32 bytes (one K-step of half a unit)
+  // weight codes: boxes of WN/2 rows x 32 bytes (one K-step of half a unit)
   if (!encode_2d_map(&P.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b, (uint64_t)(a.K / 2), (uint64_t)(a.E * a.N),
-                     BK / 2, w4::WN / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     BK / 2, WN / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const uint64_t out_cols = a.epilogue == kBfSwiGLUFwd ? (uint64_t)(a.N / 2) : (uint64_t)a.N;
   if (!encode_2d_map(&P.tmap_out, BF, 2, a.out_bf16, out_cols, (uint64_t)a.rows_cap, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   // units: at most (m-tiles + experts) / 2 pairs times the weight-row tiles
-  const int64_t units = ((a.rows_cap / BM + a.E) / 2 + 1) * (a.N / w4::WN);
+  const int64_t units = ((a.rows_cap / BM + a.E) / 2 + 1) * (a.N / WN);
   int64_t grid = num_sms();
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;
-  const size_t smem = w4::kPairsOff + 4 * (size_t)(a.E + 1) + 1024;
-  k_w4a16_gemm<<<(unsigned)grid, w4::kThreads, smem, s>>>(P);
+  const size_t smem = C::kPairsOff + 4 * (size_t)(a.E + 1) + 1024;
+  k_w4a16_gemm<C><<<(unsigned)grid, w4::kThreads, smem, s>>>(P);
   return cudaGetLastError();
+}
+
+static cudaError_t launch_w4a16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {
+  return a.w4_wide ? launch_w4a16_cfg<256>(a, s) : launch_w4a16_cfg<128>(a, s);
 }
 
 cudaError_t launch_bf16_gemm(const Bf16GemmArgs &a, cudaStream_t s) {

@@ -165,6 +165,7 @@ struct Bf16GemmArgs {
   // the per-expert decode scale applied to the accumulator in the epilogue
   const uint8_t *b_sf = nullptr;
   const float *s_dec_w = nullptr;
+  int w4_wide = 0;              // units of 256 weight rows (else 128)
   // kBfRows, K-major B (optional): the rows the A and B tensors really hold
   // (tile rows past them read as zeros), and the FP32 output's valid columns
   // and leading dimension (0: rows_cap, E * N, N and N)
