@@ -146,16 +146,6 @@ __device__ __forceinline__ void stage_row(uint32_t box_addr, int lane, const uin
     st_shared_v4(base + (((uint32_t)q ^ sw) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
 }
 
-// Group of a padded row: padded[lo] <= row < padded[lo + 1] (shared memory).
-__device__ __forceinline__ int find_group(const int32_t *padded, int E, int64_t row) {
-  int lo = 0, hi = E;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if ((int64_t)padded[mid] <= row) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
 __device__ __forceinline__ float fmax_abs_bf16(float m, uint32_t packed) {
   return fmaxf(m, fmaxf(fabsf(bf16_lo(packed)), fabsf(bf16_hi(packed))));
 }
@@ -436,16 +426,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
   const int64_t my_mtiles = m_total > (int64_t)blockIdx.x ? (m_total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const int64_t my_tiles = m_major ? my_mtiles * n_tiles
                                    : (total > (int64_t)blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0);
-  auto tile_mn = [&](int64_t i, int64_t &mt, int &nt) {
+  // The walk over the CTA's tiles advances by additions, and the m-tile's
+  // group by a short forward scan (m-tiles only grow along the walk): a
+  // division and a binary search per tile cost the epilogue warps, which
+  // redo them for every tile, a sizeable share of their time.
+  struct TileWalk {
+    int64_t mt;
+    int nt;
+    int e;
+  };
+  const int walk_dm = (int)(gridDim.x / n_tiles), walk_dn = (int)(gridDim.x % n_tiles);
+  auto walk_group = [&](TileWalk &w) {
+    while (w.e + 1 < a.E && (int64_t)s_pad[w.e + 1] <= w.mt * BM) ++w.e;
+  };
+  auto walk_start = [&]() {
+    TileWalk w;
+    w.mt = m_major ? (int64_t)blockIdx.x : (int64_t)(blockIdx.x / n_tiles);
+    w.nt = m_major ? 0 : (int)(blockIdx.x % n_tiles);
+    w.e = 0;
+    walk_group(w);
+    return w;
+  };
+  auto walk_next = [&](TileWalk &w) {
     if (m_major) {
-      const int64_t j = i / n_tiles;
-      mt = (int64_t)blockIdx.x + j * gridDim.x;
-      nt = (int)(i - j * n_tiles);
+      if (++w.nt == n_tiles) {
+        w.nt = 0;
+        w.mt += gridDim.x;
+      }
     } else {
-      const int64_t t = (int64_t)blockIdx.x + i * gridDim.x;
-      mt = t / n_tiles;
-      nt = (int)(t - mt * n_tiles);
+      w.mt += walk_dm;
+      w.nt += walk_dn;
+      if (w.nt >= n_tiles) {
+        w.nt -= n_tiles;
+        ++w.mt;
+      }
     }
+    walk_group(w);
   };
   const uint32_t steps = (uint32_t)(my_tiles * kt_count);
 
@@ -502,11 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       // step costs this thread hundreds of cycles of latency)
       uint32_t p = 0;
       bool ok = true;
-      for (int64_t i = 0; i < my_tiles && ok; ++i) {
-        int64_t mt;
-        int nt;
-        tile_mn(i, mt, nt);
-        const int e = find_group(s_pad, a.E, mt * BM);
+      TileWalk w = walk_start();
+      for (int64_t i = 0; i < my_tiles && ok; ++i, walk_next(w)) {
+        const int64_t mt = w.mt;
+        const int nt = w.nt;
+        const int e = w.e;
         const int32_t arow = (int32_t)(mt * BM);
         const int32_t wrow0 = (int32_t)((int64_t)e * a.N + (int64_t)nt * BN);
         const uint8_t *sfa_src = a.sf_a + mt * BM * 16;   // K-step 0 of the tile's rows
@@ -609,24 +625,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       }
       ++chunk_id;
     };
-    // the plain store's 32-row x 64-column box (128-byte rows, 128-byte
-    // swizzle: chunk q of row r at q ^ (r & 7)), one 4 KB buffer per warp:
-    // half the TMA store requests of two 32 x 32 boxes
-    auto store_box64 = [&](const uint32_t (&w32)[32], int32_t x, int32_t y) {
-      if (lane == 0) bulk_wait_group_read<0>();   // the buffer's previous store has read it
-      __syncwarp();
-      const uint32_t base = stg_addr + (uint32_t)lane * 128;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        st_shared_v4(base + (((uint32_t)q ^ ((uint32_t)lane & 7u)) << 4), w32[4 * q], w32[4 * q + 1], w32[4 * q + 2],
-                     w32[4 * q + 3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(&P.tmap_out, stg, x, y);
-        bulk_commit_group();
-      }
-    };
     // fused requantization: the warp's |h| maxima of a row are kept across
     // the n-tiles of an m-tile and folded into the row amax at its last
     // n-tile.  One tile later (its older bulk groups are then complete) lane
@@ -643,12 +641,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
     };
     float row_amax = 0.0f;
     bool pending_mtile = false;
-    for (int64_t i = 0; i < my_tiles; ++i, ++it) {
-      int64_t mt;
-      int nt;
-      tile_mn(i, mt, nt);
+    TileWalk w = walk_start();
+    for (int64_t i = 0; i < my_tiles; ++i, ++it, walk_next(w)) {
+      const int64_t mt = w.mt;
+      const int nt = w.nt;
       const int64_t row0 = mt * BM;
-      const int e = find_group(s_pad, a.E, row0);
+      const int e = w.e;
       const int64_t g_pad = s_pad[e];
       const int64_t g_off = s_off[e];
       const int64_t g_cnt = (int64_t)s_off[e + 1] - g_off;
@@ -760,28 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       } else {
         const int64_t orow = a.out_padded ? prow : g_off + rel;
         const int64_t col0 = (int64_t)nt * BN + half * C::kColsPerWarp;
-        if (a.out_bf16 != nullptr) {
-          const int64_t slab_row = a.out_padded ? row0 + quad * 32 : g_off + (row0 - g_pad) + quad * 32;
-#pragma unroll
-          for (int cc = 0; cc < C::kChunks / 2; ++cc) {
-            uint32_t w32[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int c = 2 * cc + (i >> 4), j = 2 * (i & 15);
-              w32[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[c][j]), scale),
-                                   __fmul_rn(__uint_as_float(v[c][j + 1]), scale));
-            }
-            if (slab_full) {
-              store_box64(w32, (int32_t)(col0 + cc * 64), (int32_t)slab_row);
-            } else if (valid) {
-              uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_bf16) +
-                                                     orow * a.N + col0 + cc * 64);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_uint4(w32[4 * q], w32[4 * q + 1], w32[4 * q + 2], w32[4 * q + 3]);
-            }
-          }
-        }
+        // FP32 first: the BF16 pass below then lets each chunk of v die as
+        // soon as it is packed, which keeps the epilogue within its registers
         if (a.out_f32 != nullptr && valid) {
           float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + orow * a.N + col0);
 #pragma unroll
@@ -792,6 +770,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
                                                __fmul_rn(__uint_as_float(v[c][i + 1]), scale),
                                                __fmul_rn(__uint_as_float(v[c][i + 2]), scale),
                                                __fmul_rn(__uint_as_float(v[c][i + 3]), scale));
+            }
+          }
+        }
+        if (a.out_bf16 != nullptr) {
+          const int64_t slab_row = a.out_padded ? row0 + quad * 32 : g_off + (row0 - g_pad) + quad * 32;
+          // 32-row x 64-column boxes (128-byte rows, 128-byte swizzle: chunk
+          // q of row r at q ^ (r & 7)) in one 4 KB buffer per warp; each
+          // 32-column half is packed and staged on its own
+          const uint32_t base = stg_addr + (uint32_t)lane * 128;
+#pragma unroll
+          for (int cc = 0; cc < C::kChunks / 2; ++cc) {
+            if (slab_full) {
+              if (lane == 0) bulk_wait_group_read<0>();   // the buffer's previous store has read it
+              __syncwarp();
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int c = 2 * cc + hh;
+              uint32_t w16[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                w16[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[c][2 * i]), scale),
+                                     __fmul_rn(__uint_as_float(v[c][2 * i + 1]), scale));
+              if (slab_full) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  st_shared_v4(base + (((uint32_t)(4 * hh + q) ^ ((uint32_t)lane & 7u)) << 4), w16[4 * q],
+                               w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+              } else if (valid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_bf16) + orow * a.N +
+                                                       col0 + cc * 64 + hh * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  dst[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+              }
+            }
+            if (slab_full) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&P.tmap_out, stg, (int32_t)(col0 + cc * 64), (int32_t)slab_row);
+                bulk_commit_group();
+              }
             }
           }
         }
