@@ -84,7 +84,7 @@ constexpr int kSlabRows = 32;
 // pieces in flight per warp.
 constexpr uint32_t kReqPiece = 5632;
 
-template <int BN_, int STAGES_, int ACC_, bool SWIGLU_, bool FUSED_ = false>
+template <int BN_, int STAGES_, int ACC_, bool SWIGLU_, bool FUSED_ = false, int STG_ = kStagingPerWarp>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr int STAGES = STAGES_;
@@ -95,6 +95,9 @@ struct Cfg {
   static constexpr bool SWIGLU = SWIGLU_;
   // with the requantization of h fused into the launch (opt-in)
   static constexpr bool FUSED = FUSED_;
+  // epilogue staging per warp: 4 KB (two 32 x 32 boxes of h, or one 32 x 64
+  // box of D), or 1 KB (one 32 x 16 box of h) to make room for a fourth stage
+  static constexpr int kStaging = STG_;
   static constexpr int kABytes = BM * BK / 2;        // 16 KB of E2M1 codes
   static constexpr int kBBytes = BN * BK / 2;
   static constexpr int kSfaBytes = BM * BK / 16;     // four 512-byte atoms
@@ -108,23 +111,27 @@ struct Cfg {
   static constexpr int kColsPerWarp = BN / 2;        // two warps share a TMEM lane quarter
   static constexpr int kChunks = kColsPerWarp / 32;
   static constexpr size_t kStagingOff = (size_t)STAGES * kStageBytes;
-  static constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStagingPerWarp;
+  static constexpr size_t kBarrierOff = kStagingOff + (size_t)kEpiWarps * kStaging;
   // fused requantization: each worker warp stages h through two buffers
   static constexpr size_t kReqOff = kBarrierOff + 512;   // barriers and flags: 512 bytes
-  static constexpr size_t kOffsetsOff = kReqOff + 4 * (size_t)kReqPiece;
+  static constexpr size_t kOffsetsOff = kReqOff + (FUSED ? 4 * (size_t)kReqPiece : 0);
   // + up to 1023 bytes lost to aligning the dynamic shared memory to 1 KB
   static constexpr size_t kSmemFixed = kOffsetsOff + 1024;
-  static constexpr size_t kSmemMax = kSmemFixed + (size_t)8 * 1025;   // + offsets of E <= 1024
+  // the group offsets (two int32 per group) take the rest: up to kMaxE groups
+  static constexpr int kMaxE = (int)((232448 - kSmemFixed) / 8) - 1;
+  static constexpr size_t kSmemMax = kSmemFixed + (size_t)8 * (kMaxE + 1);
   // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
   // UE4M3 scales (bit 23 = 0), N >> 3 at bit 17, M >> 4 at bit 24, dense, K = 64.
   static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                      ((uint32_t)(BM >> 4) << 24);
   static_assert(ACC * BN + STAGES * (16 + 16 * kNAtoms) <= (int)kTmemCols, "TMEM budget");
-  static_assert(kSmemMax <= 232448, "shared memory budget");
+  static_assert(kMaxE >= 128 && kSmemMax <= 232448, "shared memory budget");
+  static_assert(kStaging == 4096 || (kStaging == 1024 && SWIGLU && !FUSED), "staging layout");
   static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 12 <= 192, "pipeline barriers overrun their area");
 };
 
 using CfgGateUp = Cfg<256, 3, 1, true>;
+using CfgGateUp4 = Cfg<256, 4, 1, true, false, 1024>;
 using CfgGateUpFused = Cfg<256, 3, 1, true, true>;
 using CfgDown = Cfg<256, 3, 1, false>;
 
@@ -607,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
     const int half = ew >> 2;               // which half of the columns
     const int rit = quad * 32 + lane;       // row inside the tile
     const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-    uint8_t *stg = smem + C::kStagingOff + (size_t)ew * kStagingPerWarp;
+    uint8_t *stg = smem + C::kStagingOff + (size_t)ew * C::kStaging;
     const uint32_t stg_addr = smem_u32(stg);
     uint32_t chunk_id = 0;
     uint32_t it = 0;
@@ -624,6 +631,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
         bulk_commit_group();
       }
       ++chunk_id;
+    };
+    // with 1 KB of staging: a 32 x 16 box (32-byte rows, no swizzle) of 8
+    // packed words per lane, one buffer
+    auto store_box16 = [&](const uint32_t *w8, int32_t x, int32_t y) {
+      if (lane == 0) bulk_wait_group_read<0>();   // the buffer's previous store has read it
+      __syncwarp();
+      st_shared_v4(stg_addr + (uint32_t)lane * 32, w8[0], w8[1], w8[2], w8[3]);
+      st_shared_v4(stg_addr + (uint32_t)lane * 32 + 16, w8[4], w8[5], w8[6], w8[7]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&P.tmap_out, stg, x, y);
+        bulk_commit_group();
+      }
     };
     // fused requantization: the warp's |h| maxima of a row are kept across
     // the n-tiles of an m-tile and folded into the row amax at its last
@@ -701,7 +722,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
               hp[i / 2] = pack_bf16x2(hh[0], hh[1]);
               m = fmax_abs_bf16(m, hp[i / 2]);
             }
-            store_box(hp, (int32_t)(nt * 128 + half * 64 + c * 32), (int32_t)(row0 + quad * 32));
+            const int32_t hx = (int32_t)(nt * 128 + half * 64 + c * 32), hy = (int32_t)(row0 + quad * 32);
+            if constexpr (C::kStaging == 1024) {
+              store_box16(hp, hx, hy);
+              store_box16(hp + 8, hx + 16, hy);
+            } else {
+              store_box(hp, hx, hy);
+            }
           }
         };
         // the fast SwiGLU form unless some gate value of the warp's tile
@@ -830,10 +857,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
       __syncwarp();
       ReqStage rs;
       rs.buf[0] = stg;
-      rs.buf[1] = stg + kStagingPerWarp / 2;
+      rs.buf[1] = stg + C::kStaging / 2;
       rs.bar[0] = reinterpret_cast<uint64_t *>(smem + C::kBarrierOff + 224) + 2 * ew;
       rs.bar[1] = rs.bar[0] + 1;
-      rs.piece = kStagingPerWarp / 2;
+      rs.piece = C::kStaging / 2;
       rs.loads[0] = rs.loads[1] = 0;
       if (lane == 0) {
         mbar_init(rs.bar[0], 1);
@@ -926,10 +953,14 @@ cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
   if (a.out_bf16 != nullptr) {
     // D: [rows][N] (compact rows never exceed rows_cap); h: [rows_cap][N/2]
     const uint64_t cols = a.epilogue == kEpiSwiGLU ? (uint64_t)(a.N / 2) : (uint64_t)a.N;
-    // h: 32 x 32 boxes, 64-byte swizzle; D: 32 rows x 64 columns, 128-byte swizzle
+    // h: 32 x 32 boxes, 64-byte swizzle (32 x 16, none, with 1 KB of
+    // staging); D: 32 rows x 64 columns, 128-byte swizzle
     const bool wide = a.epilogue != kEpiSwiGLU;
-    if (!encode_2d(&P.tmap_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out_bf16, cols, (uint64_t)a.rows_cap,
-                   wide ? 64 : 32, 32, wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    const uint32_t box_x = wide ? 64 : (C::kStaging == 1024 ? 16 : 32);
+    const CUtensorMapSwizzle sw = wide ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : (C::kStaging == 1024 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B);
+    if (!encode_2d(&P.tmap_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out_bf16, cols, (uint64_t)a.rows_cap, box_x,
+                   32, sw))
       return cudaErrorInvalidValue;
   }
   const int64_t max_tiles = (a.rows_cap / BM) * (a.N / C::BN);
@@ -944,19 +975,24 @@ cudaError_t launch_cfg(const GemmArgs &a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
+  static_assert(CfgGateUp::kMaxE >= 1024 && CfgGateUpFused::kMaxE >= 1024 && CfgDown::kMaxE >= 1024,
+                "the three-stage kernels take every group count the library accepts");
   if (a.rows_cap <= 0) return cudaSuccess;
   // both GEMMs use 128 x 256 tiles with one accumulator (the SwiGLU epilogue
   // reads gate and up from the two 128-column halves of a tile).  128 x 128
   // tiles with two accumulators (Cfg<128, 4, 2>) also pass the parity tests
   // but run the down GEMM of the Qwen3-30B-A3B-shaped layer in 239 us
   // instead of 183 us: its cost is per K-step, not the accumulator hand-over.
-  // A fourth 54 KB stage for gate_up fits only without the epilogue's TMA
-  // staging boxes; with plain 16-byte global stores of h instead, gate_up
-  // measured 287 us against 266 us (the stage gains ~18 us, the stores lose
-  // ~39 us), so the staged 3-stage ring stays.
+  // A fourth 54 KB stage for gate_up fits when each epilogue warp stages h
+  // through one 1 KB box instead of two 2 KB ones: gate_up of that layer
+  // then takes 220 us instead of 241 us.  (With plain 16-byte global stores
+  // of h and no staging at all it was slower than three stages.)
   if (a.epilogue == kEpiSwiGLU) {
+    // gate_up: a fourth stage in the room of the epilogue's staging (1 KB
+    // boxes), as long as the group offsets of E experts still fit
     const bool fused = a.req_q != nullptr && a.amax_h != nullptr && a.amax_h_rows != 0;
-    return fused ? launch_cfg<CfgGateUpFused>(a, s) : launch_cfg<CfgGateUp>(a, s);
+    if (fused) return launch_cfg<CfgGateUpFused>(a, s);
+    return a.E <= CfgGateUp4::kMaxE ? launch_cfg<CfgGateUp4>(a, s) : launch_cfg<CfgGateUp>(a, s);
   }
   return launch_cfg<CfgDown>(a, s);
 }
