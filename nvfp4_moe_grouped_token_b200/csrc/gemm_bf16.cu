@@ -321,7 +321,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
         slab_row = (int64_t)tl.e * a.M + tl.m0 + quad * 32;
       }
       float wr = 0.0f;
-      if (a.epilogue == kBfSwiGLUBwd) wr = __ldg(a.w_rows + prow);
+      // SwiGLU backward: this lane's g and u for one 32-column chunk (row
+      // prow of G = [g | u]), loaded a chunk ahead so the loads from HBM
+      // overlap the previous chunk's arithmetic (chunk 0 before the wait)
+      const int64_t I = a.N;
+      const int64_t col0 = tl.n0 + half * 128;
+      const __nv_bfloat16 *gu = static_cast<const __nv_bfloat16 *>(a.g_u) + prow * 2 * I;
+      uint4 gq[4], uq[4];
+      auto load_gu = [&](int c) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + col0 + c * 32) + q);
+          uq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + I + col0 + c * 32) + q);
+        }
+      };
+      if (a.epilogue == kBfSwiGLUBwd) {
+        wr = __ldg(a.w_rows + prow);
+        load_gu(0);
+      }
 
       if (!mbar_wait_bounded(&acc_full[as], (it / ACC) & 1u, abort_flag, a.err, 520)) break;
       tc_fence_after();
@@ -329,8 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
       // next tile run in the other one, so this one is released after the
       // last chunk is read.  An empty expert's tile (no K-steps) is zeros.
       const bool zero_tile = tl.ksteps == 0;
-      const int64_t col0 = tl.n0 + half * 128;
-      const int64_t I = a.N;
       float dwp = 0.0f;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -377,55 +392,54 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
           //   dh = w dh', dg = dh u s (1 + g (1 - s)), du = dh g s,
           //   hw = BF16(w h), dw partial += dh' h
           const int64_t i0 = col0 + c * 32;
-          const __nv_bfloat16 *gu = static_cast<const __nv_bfloat16 *>(a.g_u) + prow * 2 * I;
           __nv_bfloat16 *dgu = static_cast<__nv_bfloat16 *>(a.d_gu) + prow * 2 * I;
           __nv_bfloat16 *hwp = static_cast<__nv_bfloat16 *>(a.hw) + prow * I;
-          uint4 gq[4], uq[4];
+          uint32_t gw[16], uw[16];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            gq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + i0) + q);
-            uq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + I + i0) + q);
+            gw[4 * q] = gq[q].x; gw[4 * q + 1] = gq[q].y; gw[4 * q + 2] = gq[q].z; gw[4 * q + 3] = gq[q].w;
+            uw[4 * q] = uq[q].x; uw[4 * q + 1] = uq[q].y; uw[4 * q + 2] = uq[q].z; uw[4 * q + 3] = uq[q].w;
           }
-          const uint32_t *gw = reinterpret_cast<const uint32_t *>(gq);
-          const uint32_t *uw = reinterpret_cast<const uint32_t *>(uq);
-          uint32_t o_dg[16], o_du[16], o_hw[16];
+          if (c < 3) load_gu(c + 1);      // the next chunk's g and u, in flight during this one
+          // eight columns at a time: compute, pack and store, so only one
+          // group's outputs are live
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float dg2[2], du2[2], hw2[2];
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o_dg[4], o_du[4], o_hw[4];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float g = q ? bf16_hi(gw[i]) : bf16_lo(gw[i]);
-              const float u = q ? bf16_hi(uw[i]) : bf16_lo(uw[i]);
-              const float dhp = __uint_as_float(v[2 * i + q]);
-              const float dh = wr * dhp;
-              // sigmoid s = sc * sp without overflow: g >= 0: sp = 1/(1+e^-g);
-              // g < 0: sp = e^g/(1+e^g); g < -64: sp = e^(g+64), sc = e^-64
-              // (then 1 + e^g and 1 - s are 1 in binary32)
-              const bool far = g < -64.0f;
-              const float t = expf(g >= 0.0f ? -g : (far ? g + 64.0f : g));
-              const float sp = (g >= 0.0f ? 1.0f : t) / (far ? 1.0f : 1.0f + t);   // one division
-              const float sc = far ? kExpM64 : 1.0f;
-              const float oms = far ? 1.0f : 1.0f - sp;
-              const float gs = g * sp;
-              const float hf = (gs * u) * sc;
-              dg2[q] = (dh * u * (sp * (1.0f + g * oms))) * sc;
-              du2[q] = (dh * gs) * sc;
-              const float h = __bfloat162float(__float2bfloat16_rn(hf));
-              hw2[q] = wr * h;
-              dwp = __fmaf_rn(dhp, h, dwp);
+            for (int j = 0; j < 4; ++j) {
+              const int i = 4 * q + j;
+              float dg2[2], du2[2], hw2[2];
+#pragma unroll
+              for (int r = 0; r < 2; ++r) {
+                const float g = r ? bf16_hi(gw[i]) : bf16_lo(gw[i]);
+                const float u = r ? bf16_hi(uw[i]) : bf16_lo(uw[i]);
+                const float dhp = __uint_as_float(v[2 * i + r]);
+                const float dh = wr * dhp;
+                // sigmoid s = sc * sp without overflow: g >= 0: sp = 1/(1+e^-g);
+                // g < 0: sp = e^g/(1+e^g); g < -64: sp = e^(g+64), sc = e^-64
+                // (then 1 + e^g and 1 - s are 1 in binary32).  Fast exponential
+                // and division (~2^-21 relative, the denominator in [1, 2]).
+                const bool far = g < -64.0f;
+                const float t = __expf(g >= 0.0f ? -g : (far ? g + 64.0f : g));
+                const float sp = __fdividef(g >= 0.0f ? 1.0f : t, far ? 1.0f : 1.0f + t);
+                const float sc = far ? kExpM64 : 1.0f;
+                const float oms = far ? 1.0f : 1.0f - sp;
+                const float gs = g * sp;
+                const float hf = (gs * u) * sc;
+                dg2[r] = (dh * u * (sp * (1.0f + g * oms))) * sc;
+                du2[r] = (dh * gs) * sc;
+                const float h = __bfloat162float(__float2bfloat16_rn(hf));
+                hw2[r] = wr * h;
+                dwp = __fmaf_rn(dhp, h, dwp);
+              }
+              o_dg[j] = pack_bf16x2(dg2[0], dg2[1]);
+              o_du[j] = pack_bf16x2(du2[0], du2[1]);
+              o_hw[j] = pack_bf16x2(hw2[0], hw2[1]);
             }
-            o_dg[i] = pack_bf16x2(dg2[0], dg2[1]);
-            o_du[i] = pack_bf16x2(du2[0], du2[1]);
-            o_hw[i] = pack_bf16x2(hw2[0], hw2[1]);
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            reinterpret_cast<uint4 *>(dgu + i0)[q] =
-                make_uint4(o_dg[4 * q], o_dg[4 * q + 1], o_dg[4 * q + 2], o_dg[4 * q + 3]);
-            reinterpret_cast<uint4 *>(dgu + I + i0)[q] =
-                make_uint4(o_du[4 * q], o_du[4 * q + 1], o_du[4 * q + 2], o_du[4 * q + 3]);
-            reinterpret_cast<uint4 *>(hwp + i0)[q] =
-                make_uint4(o_hw[4 * q], o_hw[4 * q + 1], o_hw[4 * q + 2], o_hw[4 * q + 3]);
+            reinterpret_cast<uint4 *>(dgu + i0)[q] = make_uint4(o_dg[0], o_dg[1], o_dg[2], o_dg[3]);
+            reinterpret_cast<uint4 *>(dgu + I + i0)[q] = make_uint4(o_du[0], o_du[1], o_du[2], o_du[3]);
+            reinterpret_cast<uint4 *>(hwp + i0)[q] = make_uint4(o_hw[0], o_hw[1], o_hw[2], o_hw[3]);
           }
           if (a.out_f32 != nullptr) {     // dh' itself, for inspection
             float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + prow * a.N + i0);
