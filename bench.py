@@ -348,29 +348,53 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
     ms = max_over_ranks(total_ms / steps, world, dev)
 
     # ---- end to end through the public API with host buffers ----------------
+    # Every step copies its inputs from pinned host memory and reads its whole
+    # output back.  The copies run on two copy streams with double-buffered
+    # device inputs and outputs, so step i+1's input copies and step i-1's
+    # output copy overlap step i's kernels (PCIe is full duplex).
     xh = inp["x"].pin_memory()
     ih = inp["topk_idx"].pin_memory()
     wh = inp["topk_w"].pin_memory()
-    yh = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
-    xd, idd, wd = torch.empty_like(x), torch.empty_like(idx), torch.empty_like(w)
+    yh = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    idd = [torch.empty_like(idx) for _ in range(2)]
+    wd = [torch.empty_like(w) for _ in range(2)]
+    yd = [torch.empty_like(y) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e_ in ev_in + ev_done + ev_out:
+        e_.record(stream)
 
-    def e2e_step():
-        xd.copy_(xh, non_blocking=True)
-        idd.copy_(ih, non_blocking=True)
-        wd.copy_(wh, non_blocking=True)
-        ops.moe_expert_layer(xd, idd, wd, wgu, wdn, y, ws, flags)
-        yh.copy_(y, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        s_in.wait_event(ev_done[b])              # step i-2 no longer reads input buffer b
+        with torch.cuda.stream(s_in):
+            xd[b].copy_(xh, non_blocking=True)
+            idd[b].copy_(ih, non_blocking=True)
+            wd[b].copy_(wh, non_blocking=True)
+        ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])             # step i-2's output has left buffer b
+        ops.moe_expert_layer(xd[b], idd[b], wd[b], wgu, wdn, yd[b], ws, flags)
+        ev_done[b].record(stream)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            yh[b].copy_(yd[b], non_blocking=True)
+        ev_out[b].record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = max(3, steps // 2)
-    e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(n_e2e):
+        e2e_step(i)
+    e1.record(s_out)
     torch.cuda.synchronize()
+    assert torch.equal(yh[(n_e2e - 1) % 2].view(torch.int16), yd[(n_e2e - 1) % 2].cpu().view(torch.int16))
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
 
     fl = layer_flops(cfg)
@@ -401,7 +425,9 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
                      "kernels": kern},
         "e2e": {"value": job_throughput(cfg.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4,
-                "d2h_bytes_per_step": yh.numel() * 2},
+                "d2h_bytes_per_step": yh[0].numel() * 2,
+                "pipeline": "input copies (copy stream 1), the layer (launching stream) and the output copy (copy "
+                            "stream 2) of consecutive steps overlap; double-buffered device inputs and outputs"},
         "gpu_launches": steps * launches_per_step,
         "launches_per_step": launches_per_step,
         "clocks": clk,

@@ -324,6 +324,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&p);
 }
 
+// (x0 * s, x1 * s) rounded to nearest, as one paired binary32 multiply
+// (mul.rn.f32x2: each lane of the pair is exactly __fmul_rn) packed to BF16x2.
+__device__ __forceinline__ uint32_t scale_pack_bf16x2(uint32_t x0, uint32_t x1, float s) {
+  uint64_t a, b, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "r"(x0), "r"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  float y0, y1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(d));
+  return pack_bf16x2(y0, y1);
+}
+
+// (x0 * s, x1 * s) rounded to nearest as one paired multiply, unpacked.
+__device__ __forceinline__ void scale2(uint32_t x0, uint32_t x1, float s, float &y0, float &y1) {
+  uint64_t a, b, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "r"(x0), "r"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(d));
+}
+
 // e^-64 in binary32 (a normal number).
 constexpr float kExpM64 = 1.60381089e-28f;
 

@@ -712,13 +712,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
             uint32_t hp[16];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              float hh[2];
+              float hh[2], g[2], u[2];
+              scale2(v[c][i], v[c][i + 1], scale, g[0], g[1]);
+              scale2(v[(c + 2) % C::kChunks][i], v[(c + 2) % C::kChunks][i + 1], scale, u[0], u[1]);
 #pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const float g = __fmul_rn(__uint_as_float(v[c][i + q]), scale);
-                const float u = __fmul_rn(__uint_as_float(v[(c + 2) % C::kChunks][i + q]), scale);
-                hh[q] = silu(g, u);
-              }
+              for (int q = 0; q < 2; ++q) hh[q] = silu(g[q], u[q]);
               hp[i / 2] = pack_bf16x2(hh[0], hh[1]);
               m = fmax_abs_bf16(m, hp[i / 2]);
             }
@@ -818,8 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
               uint32_t w16[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                w16[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[c][2 * i]), scale),
-                                     __fmul_rn(__uint_as_float(v[c][2 * i + 1]), scale));
+                w16[i] = scale_pack_bf16x2(v[c][2 * i], v[c][2 * i + 1], scale);
               if (slab_full) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
