@@ -20,7 +20,8 @@
 //       warp 4      TMA producer (one thread): A tile (16 KB) and B tile
 //                   (32 KB) by 128-byte-swizzled tensor copies, A's 2 KB of
 //                   K-step-major scales and B's 4 KB of scale atoms by bulk
-//                   copies, into a 3-stage shared-memory ring;
+//                   copies, into a 4-stage (gate_up, while the group
+//                   offsets still fit) or 3-stage shared-memory ring;
 //       warp 5      MMA issuer (one thread): tcgen05.mma kind::mxf4nvf4 with
 //                   16-element UE4M3 scale blocks read from TMEM, FP32
 //                   accumulation in TMEM; commits each stage back to the
@@ -30,9 +31,11 @@
 //                   accumulator (half of the columns), releases TMEM at once
 //                   so the next tile's MMAs overlap the rest of the epilogue,
 //                   scales by S_dec_a(row) * S_dec_w(expert) and stores BF16
-//                   (or FP32) rows through TMA tensor stores, or applies
-//                   SwiGLU (gate and up sit in the two 128-column halves of a
-//                   tile), stores h in BF16 and max-reduces |h| per row.
+//                   (or FP32) rows through TMA tensor stores (32 x 64
+//                   boxes), or applies SwiGLU (gate and up sit in the two
+//                   128-column halves of a tile), stores h in BF16 (32 x 32
+//                   boxes, or 32 x 16 with the 4-stage ring's 1 KB of
+//                   staging) and max-reduces |h| per row.
 //   * fused requantization (per-row scales): the CTA walks its m-tiles with
 //     all their n-tiles in a row, so a row of h -- and its amax -- is
 //     complete inside one CTA once the m-tile's last n-tile is stored.  The
@@ -46,7 +49,8 @@
 //   * persistent grid, one CTA per SM.  Without the fused requantization the
 //     CTA walks tiles t = blockIdx.x, +gridDim.x, ... over (m-tile, n-tile)
 //     with n fastest, so CTAs working at the same time share A tiles and
-//     expert weights through L2.
+//     expert weights through L2.  Every role walks its tiles by additions
+//     (the group advances by a forward scan): no per-tile division or search.
 //   * every wait is bounded (common.cuh); a timeout records an error word and
 //     the CTA drains its in-flight copies and MMAs before freeing TMEM.
 #include <cudaTypedefs.h>
@@ -74,8 +78,10 @@ constexpr int kThreads = 512;
 constexpr uint32_t kRegsFeed = 88, kRegsCtl = 72, kRegsEpi = 176;
 static_assert(128 * kRegsFeed + 128 * kRegsCtl + 256 * kRegsEpi <= 65536, "register split");
 constexpr uint32_t kTmemCols = 512;
-// Epilogue staging: per epilogue warp two 2 KB buffers of 32 rows x 32 BF16
-// (64-byte swizzle), drained to global memory by TMA tensor stores.
+// Epilogue staging per warp (default): two 2 KB buffers of 32 rows x 32 BF16
+// (64-byte swizzle) for h, or one 4 KB box of 32 x 64 (128-byte swizzle) for
+// D, drained to global memory by TMA tensor stores.  The 4-stage gate_up
+// kernel stages 1 KB per warp instead (Cfg::kStaging).
 constexpr int kStagingPerWarp = 4096;
 // Rows per slab of h: the unit of the fused requantization.
 constexpr int kSlabRows = 32;
