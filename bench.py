@@ -347,6 +347,26 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
         stage_ms.pop("requant_h")              # fused into gate_up: an empty interval
     ms = max_over_ranks(total_ms / steps, world, dev)
 
+    # ---- the same K steps replayed from one CUDA graph ----------------------
+    # (the layer makes no host synchronization or allocation, so a step
+    # captures as is; a small workload is launch-bound without it)
+    graph_ms = None
+    if world == 1:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(steps):
+                ops.moe_expert_layer(x, idx, w, wgu, wdn, y, ws, flags)
+        g.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = g0.elapsed_time(g1) / steps
+        del g
+        assert ops.device_status(ws) == 0
+
     # ---- end to end through the public API with host buffers ----------------
     # Every step copies its inputs from pinned host memory and reads its whole
     # output back.  The copies run on two copy streams with double-buffered
@@ -412,6 +432,7 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
         "stage_timing": "K further steps right after the timed ones, with a CUDA event between the kernels on the "
                         "launching stream; their mean step time is profiled_ms_per_step",
         "profiled_ms_per_step": profiled_ms,
+        "graph_ms_per_step": graph_ms,
         "step_ms_min_max": [min(step_ms), max(step_ms)],
         "roofline": {"kernel": "k_grouped_gemm (gate_up + SwiGLU epilogue)",
                      "bound": "tensor", "achieved": gu["tflops"], "peak": fp4["mma_only"], "unit": "TFLOP/s",
@@ -640,6 +661,7 @@ def run_ours(args, rank, world, local_rank):
         "stages_ms": m["stages_ms"],
         "stage_timing": m["stage_timing"],
         "profiled_ms_per_step": m["profiled_ms_per_step"],
+        "graph_ms_per_step": m["graph_ms_per_step"],
         "step_ms_min_max": m["step_ms_min_max"],
         "quantizer_gbs": next(r["gbs"] for r in m["roofline"]["kernels"] if r["stage"] == "quantize_permute"),
         "roofline": m["roofline"],
@@ -684,7 +706,8 @@ def run_ours(args, rank, world, local_rank):
             wm = measure_layer(wcfg, args, world, dev, args.workload_steps, max(3, args.warmup), fp4,
                                clocks_for_timed=False)
             extra[name] = {"workload": WORKLOAD_NAMES.get(name, name), "value": wm["value"], "unit": "tokens/s",
-                           "ms_per_step": wm["ms_per_step"], "tflops": wm["tflops"], "steps": args.workload_steps,
+                           "ms_per_step": wm["ms_per_step"], "graph_ms_per_step": wm["graph_ms_per_step"],
+                           "tflops": wm["tflops"], "steps": args.workload_steps,
                            "stages_ms": wm["stages_ms"], "roofline": wm["roofline"], "e2e": wm["e2e"],
                            "gpu_launches": wm["gpu_launches"],
                            "config": {"tokens": wcfg.T, "hidden": wcfg.H, "intermediate": wcfg.I,
