@@ -345,6 +345,19 @@ __device__ __forceinline__ void scale2(uint32_t x0, uint32_t x1, float s, float 
   asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(d));
 }
 
+// 32-byte global load (read-only path) and store; the address is 32-byte
+// aligned.
+__device__ __forceinline__ void ld_nc_v8(const void *p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st_v8(void *p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]),
+               "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // e^-64 in binary32 (a normal number).
 constexpr float kExpM64 = 1.60381089e-28f;
 

@@ -54,6 +54,11 @@ constexpr int STAGES = 4;
 constexpr int ACC = 2;
 constexpr int kThreads = 384;
 constexpr int kEpiWarp0 = 4, kEpiWarps = 8;
+// setmaxnreg: the first warpgroup (producer, MMA issuer, two idle warps)
+// gives registers to the two epilogue warpgroups: 128 * 96 + 256 * 200 =
+// 63488 of the 384 threads * 168 registers at launch.
+constexpr uint32_t kRegsCtl = 96, kRegsEpi = 200;
+static_assert(128 * kRegsCtl + 256 * kRegsEpi <= 384 * 168, "register split");
 constexpr int kABytes = BM * BK * 2;          // 16 KB
 constexpr int kBBytes = BN * BK * 2;          // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
   } else {
     total = (int64_t)a.E * m_tiles * n_tiles;
   }
-
+  if (warp < kEpiWarp0) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------- TMA producer
@@ -275,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
       mbar_wait_bounded(drain, 0, never, a.err, 512);
     }
   } else if (warp >= kEpiWarp0) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
     // -------------------------------------------------------- epilogue
     const int ew = warp - kEpiWarp0;
     const int quad = warp & 3;
@@ -327,12 +333,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
       const int64_t I = a.N;
       const int64_t col0 = tl.n0 + half * 128;
       const __nv_bfloat16 *gu = static_cast<const __nv_bfloat16 *>(a.g_u) + prow * 2 * I;
-      uint4 gq[4], uq[4];
+      // (32-byte accesses: a lane's 32 columns of g, u, dG and w h are 64
+      // bytes of its row, so each access fills whole sectors)
+      uint32_t gq[2][8], uq[2][8];
       auto load_gu = [&](int c) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          gq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + col0 + c * 32) + q);
-          uq[q] = __ldg(reinterpret_cast<const uint4 *>(gu + I + col0 + c * 32) + q);
+        for (int q = 0; q < 2; ++q) {
+          ld_nc_v8(gu + col0 + c * 32 + q * 16, gq[q]);
+          ld_nc_v8(gu + I + col0 + c * 32 + q * 16, uq[q]);
         }
       };
       if (a.epilogue == kBfSwiGLUBwd) {
@@ -396,19 +404,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
           __nv_bfloat16 *hwp = static_cast<__nv_bfloat16 *>(a.hw) + prow * I;
           uint32_t gw[16], uw[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            gw[4 * q] = gq[q].x; gw[4 * q + 1] = gq[q].y; gw[4 * q + 2] = gq[q].z; gw[4 * q + 3] = gq[q].w;
-            uw[4 * q] = uq[q].x; uw[4 * q + 1] = uq[q].y; uw[4 * q + 2] = uq[q].z; uw[4 * q + 3] = uq[q].w;
+          for (int j = 0; j < 8; ++j) {
+            gw[j] = gq[0][j]; gw[8 + j] = gq[1][j];
+            uw[j] = uq[0][j]; uw[8 + j] = uq[1][j];
           }
           if (c < 3) load_gu(c + 1);      // the next chunk's g and u, in flight during this one
-          // eight columns at a time: compute, pack and store, so only one
+          // sixteen columns at a time: compute, pack and store, so only one
           // group's outputs are live
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t o_dg[4], o_du[4], o_hw[4];
+          for (int q = 0; q < 2; ++q) {
+            uint32_t o_dg[8], o_du[8], o_hw[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int i = 4 * q + j;
+            for (int j = 0; j < 8; ++j) {
+              const int i = 8 * q + j;
               float dg2[2], du2[2], hw2[2];
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
@@ -437,9 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
               o_du[j] = pack_bf16x2(du2[0], du2[1]);
               o_hw[j] = pack_bf16x2(hw2[0], hw2[1]);
             }
-            reinterpret_cast<uint4 *>(dgu + i0)[q] = make_uint4(o_dg[0], o_dg[1], o_dg[2], o_dg[3]);
-            reinterpret_cast<uint4 *>(dgu + I + i0)[q] = make_uint4(o_du[0], o_du[1], o_du[2], o_du[3]);
-            reinterpret_cast<uint4 *>(hwp + i0)[q] = make_uint4(o_hw[0], o_hw[1], o_hw[2], o_hw[3]);
+            st_v8(dgu + i0 + q * 16, o_dg);
+            st_v8(dgu + I + i0 + q * 16, o_du);
+            st_v8(hwp + i0 + q * 16, o_hw);
           }
           if (a.out_f32 != nullptr) {     // dh' itself, for inspection
             float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + prow * a.N + i0);
