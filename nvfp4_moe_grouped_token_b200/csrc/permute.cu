@@ -83,15 +83,17 @@ __global__ void __launch_bounds__(kRankTokens) k_route_count(const PermuteParams
   }
   __syncthreads();
   if (live) {
-    // plain (coherent) loads: the fused variant wrote these ids in this launch
+    // the fused variant wrote these ids in this launch: coherent loads there;
+    // given ids are read-only here and sit in L1 since the first pass
     const int32_t *row = p.topk_idx + t * k;
+    auto id_at = [&](int j) { return NE > 0 ? __ldcg(row + j) : __ldg(row + j); };
     const uint32_t below = (1u << lane) - 1u;
     for (int j = 0; j < k; ++j) {
-      const int e = __ldcg(row + j);
+      const int e = id_at(j);
       int32_t r = -1;
       if (e >= 0 && e < E) {
         bool dup = false;
-        for (int jj = 0; jj < j; ++jj) dup |= (__ldcg(row + jj) == e);
+        for (int jj = 0; jj < j; ++jj) dup |= (id_at(jj) == e);
         if (!dup) r = wpre[warp * E + e] + __popc(masks[warp * E + e] & below);
       }
       p.local_rank[t * k + j] = r;
@@ -110,9 +112,18 @@ __global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams
   const int64_t seg = (nblk + S - 1) / S;
   const int64_t b0 = (int64_t)s * seg;
   const int64_t b1 = b0 + seg < nblk ? b0 + seg : nblk;
+  // eight loads in flight per step: one at a time, the segment's loads would
+  // each wait out a full memory latency
+  constexpr int kBatch = 8;
   int32_t sum = 0;
   if (s < S) {
-    for (int64_t b = b0; b < b1; ++b) sum += p.block_counts[b * E + e];
+    for (int64_t b = b0; b < b1; b += kBatch) {
+      int32_t c[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) c[j] = b + j < b1 ? p.block_counts[(b + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) sum += c[j];
+    }
     partial[s * E + e] = sum;
   }
   __syncthreads();
@@ -124,10 +135,15 @@ __global__ void __launch_bounds__(kScanThreads) k_route_scan(const PermuteParams
       if (ss < s) base += v;
       total += v;
     }
-    for (int64_t b = b0; b < b1; ++b) {
-      const int32_t c = p.block_counts[b * E + e];
-      p.block_counts[b * E + e] = base;
-      base += c;
+    for (int64_t b = b0; b < b1; b += kBatch) {
+      int32_t c[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) c[j] = b + j < b1 ? p.block_counts[(b + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (b + j < b1) p.block_counts[(b + j) * E + e] = base;
+        base += c[j];
+      }
     }
   }
   // inclusive scans of totals and padded totals over experts: a warp scan,
