@@ -769,6 +769,7 @@ int moe_expert_layer_backward(const void *x, const int32_t *topk_idx, const floa
   gp.topk_w = topk_w;
   gp.topk_idx = topk_idx;
   gp.perm = perm;
+  gp.inv_perm = inv_perm;
   gp.offsets = offsets;
   gp.padded_offsets = padded;
   gp.T = T;
@@ -979,6 +980,7 @@ int w4ax_layer(const void *x, const int32_t *topk_idx, const float *topk_w, cons
   gp.topk_w = topk_w;
   gp.topk_idx = topk_idx;
   gp.perm = perm;
+  gp.inv_perm = inv_perm;
   gp.offsets = offsets;
   gp.padded_offsets = padded;
   gp.T = T;

@@ -207,6 +207,7 @@ struct BwdGatherParams {
   const void *x, *dy;
   const float *topk_w;
   const int32_t *topk_idx, *perm, *offsets, *padded_offsets;
+  const int32_t *inv_perm;   // [T][k] compact row of each (token, slot), -1 if unrouted
   int64_t T, H, rows_cap;
   int k, E;
   void *x_rows, *dy_rows;
