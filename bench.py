@@ -295,10 +295,18 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
     assert ops.device_status(ws) == 0
 
     # ---- timed region: K steps through the public API, inputs resident in
-    # HBM; then K more steps with a CUDA event between the kernels for the
-    # stage times (an event record between two kernels costs the step a few
-    # microseconds, so those steps are not the ones timed)
+    # HBM, with CUDA events only around the gate_up GEMM (the roofline's
+    # kernel); then K more steps with an event between every two kernels for
+    # the stage breakdown (each event record costs a step a few microseconds,
+    # so the timed steps carry two)
     nstage = len(ops.STAGES)
+    gu_stage = ops.STAGES.index("gate_up_swiglu")
+    gu_evs = [[None] * (nstage + 1) for _ in range(steps)]
+    for row in gu_evs:
+        row[gu_stage] = torch.cuda.Event(enable_timing=True)
+        row[gu_stage + 1] = torch.cuda.Event(enable_timing=True)
+        row[gu_stage].record(stream)
+        row[gu_stage + 1].record(stream)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(steps)]
     for row in evs:                          # materialise the events before timing
         for e in row:
@@ -317,7 +325,7 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
         clocks.mark_begin()
     t_start.record(stream)
     for i in range(steps):
-        ops.moe_expert_layer(x, idx, w, wgu, wdn, y, ws, flags)
+        ops.moe_expert_layer_profiled(x, idx, w, wgu, wdn, y, ws, gu_evs[i], flags)
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -345,6 +353,9 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
                 for j, name in enumerate(ops.STAGES)}
     if flags & FUSED_REQUANT_FLAG:
         stage_ms.pop("requant_h")              # fused into gate_up: an empty interval
+    # the roofline kernel's time from the timed steps themselves
+    gate_up_timed_ms = statistics.mean(gu_evs[i][gu_stage].elapsed_time(gu_evs[i][gu_stage + 1])
+                                       for i in range(steps))
     ms = max_over_ranks(total_ms / steps, world, dev)
 
     # ---- the same K steps replayed from one CUDA graph ----------------------
@@ -421,7 +432,7 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
     pk = peaks()
     traffic = load_traffic("gate_up_swiglu") if cfg.name == "moe30b" else None
     kern = kernel_rooflines(cfg, stage_ms, args.per_tensor, pk, fp4, traffic, bool(flags & FUSED_REQUANT_FLAG))
-    gu = next(r for r in kern if r["stage"] == "gate_up_swiglu")
+    gu_tflops = fl["gate_up"] / (gate_up_timed_ms * 1e-3) / 1e12
     bf16x4 = pk["bf16_tflops"] * FP4_PER_BF16
     launches_per_step = 7 + (1 if args.per_tensor else 0) - (1 if flags & FUSED_REQUANT_FLAG else 0)
     return {
@@ -435,14 +446,16 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
         "graph_ms_per_step": graph_ms,
         "step_ms_min_max": [min(step_ms), max(step_ms)],
         "roofline": {"kernel": "k_grouped_gemm (gate_up + SwiGLU epilogue)",
-                     "bound": "tensor", "achieved": gu["tflops"], "peak": fp4["mma_only"], "unit": "TFLOP/s",
-                     "frac": gu["tflops"] / fp4["mma_only"], "traffic": traffic,
+                     "bound": "tensor", "achieved": gu_tflops, "peak": fp4["mma_only"], "unit": "TFLOP/s",
+                     "frac": gu_tflops / fp4["mma_only"], "traffic": traffic,
+                     "kernel_ms": gate_up_timed_ms,
+                     "kernel_timing": "CUDA events around the kernel in every timed step, on its launching stream",
                      "peak_note": "block-scaled FP4 MMA (M128 N256 K64) measured in this process, operands in "
                                   "shared memory (nvfp4moe_mma_peak)",
                      "peak_with_scale_writes": fp4["with_scale_writes"],
-                     "frac_vs_bf16_burst_x4": gu["tflops"] / bf16x4,
+                     "frac_vs_bf16_burst_x4": gu_tflops / bf16x4,
                      "bf16_burst_x4": bf16x4, "bf16_source": pk["source"],
-                     "frac_vs_nominal_9pf": gu["tflops"] / 9000.0,
+                     "frac_vs_nominal_9pf": gu_tflops / 9000.0,
                      "kernels": kern},
         "e2e": {"value": job_throughput(cfg.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4,

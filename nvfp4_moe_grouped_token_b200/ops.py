@@ -418,14 +418,15 @@ STAGES = ["route", "quantize_permute", "gate_up_swiglu", "requant_h", "down", "c
 def moe_expert_layer_profiled(x, topk_idx, topk_w, w_gate_up: NVFP4Weights, w_down: NVFP4Weights, y,
                               workspace, events, flags=0, stream=None):
     """moe_expert_layer recording the 7 torch.cuda.Event objects in `events`
-    (created with enable_timing=True) at the stage boundaries."""
+    (created with enable_timing=True) at the stage boundaries; a None entry
+    records nothing there."""
     _dev(x, topk_idx, topk_w, y, workspace)
     T, H = x.shape
     k = topk_idx.shape[1]
     I = w_down.K
     arr = (ctypes.c_void_p * 7)()
     for i, ev in enumerate(events):
-        arr[i] = ctypes.c_void_p(ev.cuda_event)
+        arr[i] = None if ev is None else ctypes.c_void_p(ev.cuda_event)
     gu, dn = w_gate_up.struct(), w_down.struct()
     _check(lib().moe_expert_layer_profiled(_p(x), _p(topk_idx), _p(topk_w), ctypes.byref(gu),
                                            ctypes.byref(dn), T, H, I, w_down.E, k, _p(y), flags,

@@ -291,3 +291,32 @@ def test_layer_replays_from_a_cuda_graph():
         assert ops.device_status(L.ws) == 0
         assert torch.equal(y_graph.view(torch.int16), y_eager.view(torch.int16))
     del g
+
+
+def test_moe30b_exact_stages_every_row():
+    """The bit-exact stages on every routed row of the Qwen3-30B-A3B-shaped
+    layer (per-token scaling, as benched): the x codes, scales and S_dec
+    scattered to all 131072 rows, and the requantization of the GPU's h (amax
+    from the epilogue) on all of them."""
+    cfg = workloads.CONFIGS["moe30b"]
+    L = Layer(cfg, ops.SCALE_PER_TOKEN)
+    L.run()
+    T, H, I, k = cfg.T, cfg.H, cfg.I, cfg.k
+    v = L.v
+    info = cpp.permutation(L.inp["topk_idx"].numpy(), cfg.E)
+    for key in ("offsets", "padded_offsets", "perm"):
+        assert np.array_equal(v[key].cpu().numpy(), info[key]), key
+    prow = padded_rows(info)
+    tok = info["perm"] // k
+    cap = v["rows_cap"]
+    qx = cpp.quantize(L.inp["x"].float().numpy(), True)
+    xq = v["x_q"].cpu().numpy()[prow]
+    xsf = ops.sf_kstep_to_rowmajor(v["x_sf"].cpu(), cap, H).numpy()[prow]
+    assert np.array_equal(xq, qx["q"][tok])
+    assert np.array_equal(xsf, qx["sf"][tok])
+    assert np.array_equal(v["x_sdec"].cpu().numpy()[prow], qx["s_dec"][tok])
+    h = v["h"].float().cpu().numpy()[prow]
+    qh = cpp.quantize(h, True)
+    assert np.array_equal(v["h_q"].cpu().numpy()[prow], qh["q"])
+    assert np.array_equal(ops.sf_kstep_to_rowmajor(v["h_sf"].cpu(), cap, I).numpy()[prow], qh["sf"])
+    assert np.array_equal(v["h_sdec"].cpu().numpy()[prow], qh["s_dec"])
