@@ -326,25 +326,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
         orow = (int64_t)tl.e * a.M + tl.m0 + quad * 32 + lane;
         slab_row = (int64_t)tl.e * a.M + tl.m0 + quad * 32;
       }
-      float wr = 0.0f;
-      // SwiGLU backward: this lane's g and u for one 32-column chunk (row
-      // prow of G = [g | u]), loaded a chunk ahead so the loads from HBM
-      // overlap the previous chunk's arithmetic (chunk 0 before the wait)
+      // SwiGLU backward, processed transposed: each 32 x 32 chunk of dh'
+      // goes through the warp's staging tile in shared memory, and lane l
+      // then takes rows rl + 8 k (k < 4, rl = l / 4) of the warp's 32 and
+      // columns 8 s .. 8 s + 7 (s = l % 4) of the chunk.  Every global access
+      // of the chunk (g, u, dG, w h) then covers 8 rows x 64 contiguous bytes
+      // instead of one row per lane.  g and u are loaded a chunk ahead, so
+      // their HBM latency overlaps the previous chunk (chunk 0 before the
+      // accumulator wait).
       const int64_t I = a.N;
       const int64_t col0 = tl.n0 + half * 128;
-      const __nv_bfloat16 *gu = static_cast<const __nv_bfloat16 *>(a.g_u) + prow * 2 * I;
-      // (32-byte accesses: a lane's 32 columns of g, u, dG and w h are 64
-      // bytes of its row, so each access fills whole sectors)
-      uint32_t gq[2][8], uq[2][8];
+      const int s4 = lane & 3, rl = lane >> 2;
+      const int64_t prow_t0 = tl.m0 + quad * 32 + rl;     // row of k = 0; k adds 8 k
+      uint4 gq[4], uq[4];
       auto load_gu = [&](int c) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          ld_nc_v8(gu + col0 + c * 32 + q * 16, gq[q]);
-          ld_nc_v8(gu + I + col0 + c * 32 + q * 16, uq[q]);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const __nv_bfloat16 *gr = static_cast<const __nv_bfloat16 *>(a.g_u) + (prow_t0 + 8 * k4) * 2 * I +
+                                    col0 + c * 32 + 8 * s4;
+          gq[k4] = __ldg(reinterpret_cast<const uint4 *>(gr));
+          uq[k4] = __ldg(reinterpret_cast<const uint4 *>(gr + I));
         }
       };
+      float wr_t[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       if (a.epilogue == kBfSwiGLUBwd) {
-        wr = __ldg(a.w_rows + prow);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) wr_t[k4] = __ldg(a.w_rows + prow_t0 + 8 * k4);
         load_gu(0);
       }
 
@@ -354,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
       // next tile run in the other one, so this one is released after the
       // last chunk is read.  An empty expert's tile (no K-steps) is zeros.
       const bool zero_tile = tl.ksteps == 0;
-      float dwp = 0.0f;
+      float dwp_t[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // <dh', h> of rows rl + 8 k over this lane's columns
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
@@ -395,34 +402,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
                                        __uint_as_float(v[i + 3]));
           }
         } else {
-          // SwiGLU backward, padded row prow, columns i0 .. i0+31 of I:
+          // SwiGLU backward, columns i0 .. i0+31 of I:
           //   dh' = accumulator (dy W_dn), s = sigmoid(g), h = BF16(g s u),
           //   dh = w dh', dg = dh u s (1 + g (1 - s)), du = dh g s,
           //   hw = BF16(w h), dw partial += dh' h
           const int64_t i0 = col0 + c * 32;
-          __nv_bfloat16 *dgu = static_cast<__nv_bfloat16 *>(a.d_gu) + prow * 2 * I;
-          __nv_bfloat16 *hwp = static_cast<__nv_bfloat16 *>(a.hw) + prow * I;
-          uint32_t gw[16], uw[16];
+          if (a.out_f32 != nullptr) {     // dh' itself, for inspection (lane = row prow)
+            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + prow * a.N + i0);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            gw[j] = gq[0][j]; gw[8 + j] = gq[1][j];
-            uw[j] = uq[0][j]; uw[8 + j] = uq[1][j];
+            for (int i = 0; i < 32; i += 4)
+              dst[i / 4] = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                       __uint_as_float(v[i + 3]));
           }
-          if (c < 3) load_gu(c + 1);      // the next chunk's g and u, in flight during this one
-          // sixteen columns at a time: compute, pack and store, so only one
-          // group's outputs are live
+          // the chunk into the staging tile: 16-byte piece m of row `lane` at
+          // piece m ^ (lane & 7) (conflict-free both ways)
+          const uint32_t trow = stg_addr + (uint32_t)lane * 128;
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t o_dg[8], o_du[8], o_hw[8];
+          for (int m = 0; m < 8; ++m)
+            st_shared_v4(trow + (((uint32_t)m ^ ((uint32_t)lane & 7u)) << 4), v[4 * m], v[4 * m + 1], v[4 * m + 2],
+                         v[4 * m + 3]);
+          __syncwarp();
+          uint4 dq[4][2];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int i = 8 * q + j;
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint32_t r = (uint32_t)(rl + 8 * k4);
+            const uint32_t rb = stg_addr + r * 128;
+            dq[k4][0] = ld_shared_v4(rb + (((uint32_t)(2 * s4) ^ (r & 7u)) << 4));
+            dq[k4][1] = ld_shared_v4(rb + (((uint32_t)(2 * s4 + 1) ^ (r & 7u)) << 4));
+          }
+          __syncwarp();                         // the tile is free for the next chunk
+          uint4 gc[4], uc[4];
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            gc[k4] = gq[k4];
+            uc[k4] = uq[k4];
+          }
+          if (c < 3) load_gu(c + 1);           // the next chunk's g and u, in flight during this one
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint32_t gw[4] = {gc[k4].x, gc[k4].y, gc[k4].z, gc[k4].w};
+            const uint32_t uw[4] = {uc[k4].x, uc[k4].y, uc[k4].z, uc[k4].w};
+            const uint32_t dw[8] = {dq[k4][0].x, dq[k4][0].y, dq[k4][0].z, dq[k4][0].w,
+                                    dq[k4][1].x, dq[k4][1].y, dq[k4][1].z, dq[k4][1].w};
+            const float wr = wr_t[k4];
+            uint32_t o_dg[4], o_du[4], o_hw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
               float dg2[2], du2[2], hw2[2];
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
                 const float g = r ? bf16_hi(gw[i]) : bf16_lo(gw[i]);
                 const float u = r ? bf16_hi(uw[i]) : bf16_lo(uw[i]);
-                const float dhp = __uint_as_float(v[2 * i + r]);
+                const float dhp = __uint_as_float(dw[2 * i + r]);
                 const float dh = wr * dhp;
                 // sigmoid s = sc * sp without overflow: g >= 0: sp = 1/(1+e^-g);
                 // g < 0: sp = e^g/(1+e^g); g < -64: sp = e^(g+64), sc = e^-64
@@ -439,26 +470,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
                 du2[r] = (dh * gs) * sc;
                 const float h = __bfloat162float(__float2bfloat16_rn(hf));
                 hw2[r] = wr * h;
-                dwp = __fmaf_rn(dhp, h, dwp);
+                dwp_t[k4] = __fmaf_rn(dhp, h, dwp_t[k4]);
               }
-              o_dg[j] = pack_bf16x2(dg2[0], dg2[1]);
-              o_du[j] = pack_bf16x2(du2[0], du2[1]);
-              o_hw[j] = pack_bf16x2(hw2[0], hw2[1]);
+              o_dg[i] = pack_bf16x2(dg2[0], dg2[1]);
+              o_du[i] = pack_bf16x2(du2[0], du2[1]);
+              o_hw[i] = pack_bf16x2(hw2[0], hw2[1]);
             }
-            st_v8(dgu + i0 + q * 16, o_dg);
-            st_v8(dgu + I + i0 + q * 16, o_du);
-            st_v8(hwp + i0 + q * 16, o_hw);
-          }
-          if (a.out_f32 != nullptr) {     // dh' itself, for inspection
-            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + prow * a.N + i0);
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              dst[i / 4] = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
-                                       __uint_as_float(v[i + 3]));
+            const int64_t pr = prow_t0 + 8 * k4;
+            __nv_bfloat16 *dgu = static_cast<__nv_bfloat16 *>(a.d_gu) + pr * 2 * I + i0 + 8 * s4;
+            __nv_bfloat16 *hwp = static_cast<__nv_bfloat16 *>(a.hw) + pr * I + i0 + 8 * s4;
+            *reinterpret_cast<uint4 *>(dgu) = make_uint4(o_dg[0], o_dg[1], o_dg[2], o_dg[3]);
+            *reinterpret_cast<uint4 *>(dgu + I) = make_uint4(o_du[0], o_du[1], o_du[2], o_du[3]);
+            *reinterpret_cast<uint4 *>(hwp) = make_uint4(o_hw[0], o_hw[1], o_hw[2], o_hw[3]);
           }
         }
       }
-      if (a.epilogue == kBfSwiGLUBwd) a.dw_part[prow * (I / 128) + (col0 / 128)] = dwp;
+      if (a.epilogue == kBfSwiGLUBwd) {
+        // each row's partial over the warp's 128 columns: the four lanes of
+        // the row (s = 0..3) hold 32 columns each
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          float d = dwp_t[k4];
+          d += __shfl_xor_sync(0xffffffffu, d, 1);
+          d += __shfl_xor_sync(0xffffffffu, d, 2);
+          if (s4 == 0) a.dw_part[(prow_t0 + 8 * k4) * (I / 128) + (col0 / 128)] = d;
+        }
+      }
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
@@ -621,12 +658,6 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
-}
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
-  return v;
 }
 
 __device__ __forceinline__ uint32_t ld_shared_u16(uint32_t saddr) {
