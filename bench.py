@@ -419,7 +419,7 @@ def measure_layer(cfg, args, world, dev, steps, warmup, fp4, clocks_for_timed=Tr
         e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(3, steps // 2)
+    n_e2e = max(3, steps)
     e0.record(s_in)
     for i in range(n_e2e):
         e2e_step(i)
