@@ -367,11 +367,33 @@ __device__ __forceinline__ void st_v8(void *p, const uint32_t (&r)[8]) {
 // e^-64 in binary32 (a normal number).
 constexpr float kExpM64 = 1.60381089e-28f;
 
-// silu(g) * u, the fast form g / (1 + e^-g) * u (fast exponential and
-// division, ~2^-21 relative): valid for g >= -64 (near g = -87 e^-g leaves
-// the fast division's range, 2^126, and the quotient flushes to zero).
-__device__ __forceinline__ float silu_mul_fast(float g, float u) {
-  return __fmul_rn(__fdividef(g, 1.0f + __expf(-g)), u);
+// silu(g) u for a pair (g0, u0), (g1, u1) with g >= -64: g / (1 + 2^(-g
+// log2 e)) u from the MUFU's approximate base-2 exponential and reciprocal
+// (ex2.approx / rcp.approx, a few ulp), the multiplies and the add paired
+// (f32x2).  Beyond g = 87 the exponential flushes to 0 and h = g u; at
+// g = -64 the denominator is 2^92, inside the reciprocal's range.
+__device__ __forceinline__ void silu_mul_fast2(float g0, float g1, float u0, float u1, float &h0, float &h1) {
+  constexpr float kNegLog2e = -1.44269504088896340736f;
+  uint64_t gg, ll, x, d, one, r, q, uu, hh;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(gg) : "f"(g0), "f"(g1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(ll) : "f"(kNegLog2e));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(x) : "l"(gg), "l"(ll));
+  float x0, x1, e0, e1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(x0));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(x1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(e0), "f"(e1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(one) : "f"(1.0f));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(d), "l"(one));
+  float d0, d1, r0, r1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(d0));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(d1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(r0), "f"(r1));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q) : "l"(gg), "l"(r));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(uu) : "f"(u0), "f"(u1));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(hh) : "l"(q), "l"(uu));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(h0), "=f"(h1) : "l"(hh));
 }
 
 // silu(g) * u in binary32 with one fast exponential and one fast division

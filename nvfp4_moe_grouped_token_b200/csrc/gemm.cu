@@ -712,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
         // the group's end are padding that nothing reads); each 32-column
         // chunk is stored as soon as it is computed, which keeps the
         // epilogue's registers within its share
-        auto swiglu = [&](auto silu) {
+        auto swiglu = [&](auto silu2) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t hp[16];
@@ -721,8 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
               float hh[2], g[2], u[2];
               scale2(v[c][i], v[c][i + 1], scale, g[0], g[1]);
               scale2(v[(c + 2) % C::kChunks][i], v[(c + 2) % C::kChunks][i + 1], scale, u[0], u[1]);
-#pragma unroll
-              for (int q = 0; q < 2; ++q) hh[q] = silu(g[q], u[q]);
+              silu2(g[0], g[1], u[0], u[1], hh[0], hh[1]);
               hp[i / 2] = pack_bf16x2(hh[0], hh[1]);
               m = fmax_abs_bf16(m, hp[i / 2]);
             }
@@ -743,9 +742,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_gemm(const __grid_const
 #pragma unroll
           for (int i = 0; i < 32; ++i) gmin = fminf(gmin, __uint_as_float(v[c][i]));
         if (__any_sync(0xffffffffu, __fmul_rn(gmin, scale) < -64.0f))
-          swiglu([](float g, float u) { return silu_mul(g, u); });
+          swiglu([](float g0, float g1, float u0, float u1, float &h0, float &h1) {
+            h0 = silu_mul(g0, u0);
+            h1 = silu_mul(g1, u1);
+          });
         else
-          swiglu([](float g, float u) { return silu_mul_fast(g, u); });
+          swiglu([](float g0, float g1, float u0, float u1, float &h0, float &h1) {
+            silu_mul_fast2(g0, g1, u0, u1, h0, h1);
+          });
         if (a.amax_h != nullptr) {
           if (a.amax_h_rows) {
             if (!fused_requant) {
