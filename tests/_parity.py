@@ -4,7 +4,7 @@ The reference values come from the plain C++ oracle (oracle/nvfp4_oracle.cpp
 through oracle.cpp); index helpers (padded row positions, the expert of a
 sorted row, BF16 spacing) are plain numpy here.
 
-Tolerances (benchmark spec of the problem):
+Tolerances (the statement of the problem):
   * codes, scales, amax, S_dec, offsets and permutation: bit-exact;
   * a GEMM output in FP32: |gpu - exact| <= 1e-5 * sum_k |a_k w_k| + 1e-6;
   * a BF16 output: within one BF16 ulp of the exact value rounded to BF16,

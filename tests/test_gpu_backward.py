@@ -2,7 +2,7 @@
 
 Stage by stage and teacher-forced: each GPU stage is recomputed by the C++
 oracle from the GPU's own stored inputs (BF16 rows, G, dG, w*h, dh'), with the
-the benchmark spec's GEMM tolerance |err| <= 1e-5 * sum|a b| + 1e-6 in FP32 and one
+stated GEMM tolerance |err| <= 1e-5 * sum|a b| + 1e-6 in FP32 and one
 BF16 ulp for BF16 outputs; the elementwise SwiGLU backward with a bound derived
 from its FP32 arithmetic.  End to end, the gradients are compared with the
 oracle's exact fp64 gradient of the unquantized layer (R16); BF16 storage of
