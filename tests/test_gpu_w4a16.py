@@ -2,7 +2,7 @@
 weights as the W4A4 layer (converted to BF16 tile by tile inside the GEMM).
 
 Stage by stage and teacher-forced against the C++ oracle: each GPU stage is
-recomputed from the GPU's own previous-stage output with the benchmark spec's
+recomputed from the GPU's own previous-stage output with the stated
 GEMM tolerance (1e-5 * sum|a w| + 1e-6 in FP32, then one BF16 ulp); the
 permutation and the gathered rows are exact.  The whole layer is also
 compared with the oracle's W4A16 layer (R19)."""

@@ -4,7 +4,7 @@ are exact in BF16).
 
 Teacher-forced against the C++ oracle: the MXFP8 quantize-dequantize of x
 and of the GPU's own BF16 h are bit-exact; h before its requantization, D and
-y are within the benchmark spec's GEMM tolerance (1e-5 * sum|a w| + 1e-6 in FP32,
+y are within the stated GEMM tolerance (1e-5 * sum|a w| + 1e-6 in FP32,
 then one BF16 ulp).  The whole layer is also compared with the oracle's W4A8
 layer (R20)."""
 import numpy as np
