@@ -69,13 +69,13 @@ constexpr int BM = 128, BK = 256;
 // 16 warps in four warpgroups: 0-3 scale feeders (one per TMEM lane quarter),
 // 4 the TMA producer, 5 the MMA issuer, 6-7 the requantization workers, 8-15
 // the epilogue.  setmaxnreg moves registers from the first two warpgroups to
-// the epilogue: 128 * 88 + 128 * 72 + 256 * 176 = 65536 launched (512 * 128).
+// the epilogue: 128 * 80 + 128 * 64 + 256 * 184 = 65536 launched (512 * 128).
 constexpr int kFeedWarps = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 8;
 constexpr int kWorkWarp0 = 6;
 constexpr int kThreads = 512;
-constexpr uint32_t kRegsFeed = 88, kRegsCtl = 72, kRegsEpi = 176;
+constexpr uint32_t kRegsFeed = 80, kRegsCtl = 64, kRegsEpi = 184;
 static_assert(128 * kRegsFeed + 128 * kRegsCtl + 256 * kRegsEpi <= 65536, "register split");
 constexpr uint32_t kTmemCols = 512;
 // Epilogue staging per warp (default): two 2 KB buffers of 32 rows x 32 BF16
