@@ -25,7 +25,11 @@
 //   * K-step of 64 elements, a 4-stage ring (A 16 KB + B 32 KB per stage).
 //   * warp 0: TMA producer (one thread); warp 1: TMEM owner and MMA issuer
 //     (one thread); warps 4-11: epilogue, two per TMEM lane quarter, each
-//     reading half of the 256 columns.
+//     reading half of the 256 columns (setmaxnreg: 200 registers for the
+//     epilogue warpgroups, 96 for the first).  BF16 outputs leave through
+//     TMA tensor stores; the SwiGLU-backward epilogue instead runs each 32 x
+//     32 chunk transposed through the warp's staging tile, so its loads of g
+//     and u and its stores of dG and w h cover 8 rows x 64 bytes each.
 //   * kBfRows: tiles over (m-tile, n-tile) of the padded grouped rows with n
 //     fastest; the expert of an m-tile comes from padded_offsets.
 //     kBfWgrad: tiles over (expert, m-tile, n-tile); the K loop covers the
