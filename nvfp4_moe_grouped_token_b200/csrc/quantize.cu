@@ -397,7 +397,9 @@ cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
     // every padded row below rows_cap, every block; 32-bit indices
     if (p.rows_cap * (int64_t)nblk >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     int64_t blocks = (p.rows_cap * nblk + 255) / 256;
-    const int64_t persistent = (int64_t)num_sms() * 8;  // 8 CTAs of 256 threads per SM
+    // 16 CTAs of 256 threads per SM (two waves of 8): measured 4-5 us faster on
+    // the moe30b layer than one resident wave of 8, and 4 per SM slower
+    const int64_t persistent = (int64_t)num_sms() * 16;
     if (blocks > persistent) blocks = persistent;
     if (blocks < 1) blocks = 1;
     k_requant_blocks<<<(unsigned)blocks, 256, 0, s>>>(p, nblk);
