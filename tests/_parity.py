@@ -153,6 +153,8 @@ def dequant_weights(prep, e: int, gate_up: bool) -> np.ndarray:
 def swiglu_bound(g, u, tg, tu):
     """Bound on |silu(g')u' - silu(g)u| for |g'-g| <= tg, |u'-u| <= tu
     (|silu'| <= 1.1), plus FP32 epilogue rounding (a few ulps of h)."""
-    s = np.abs(g / (1.0 + np.exp(-np.asarray(g, dtype=np.float64))))
+    g64 = np.asarray(g, dtype=np.float64)
+    # exp is clipped where silu(g) is already below any float: no overflow warning
+    s = np.abs(g64 / (1.0 + np.exp(np.minimum(-g64, 700.0))))
     h = np.abs(s * u)
     return 1.1 * tg * (np.abs(u) + tu) + (s + 1.1 * tg) * tu + 8 * 2.0 ** -24 * h + 1e-30
