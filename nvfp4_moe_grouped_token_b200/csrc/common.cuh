@@ -74,20 +74,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of the same condition (try_wait may suspend the thread
-// for a while; a polling loop that serves two roles must not).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for the phase with the given parity to complete.  Gives up when
 // *abort becomes nonzero or after kWaitTimeoutNs (then records kDevTimeout in
 // err, raises *abort, and returns false).  Never spins without a bound.
@@ -218,13 +204,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Copy one 512-byte scale-factor atom (32 rows x 128 bits) from shared memory
-// into TMEM lanes 0..31, replicated into all four 32-lane sub-partitions.
-__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
 // D[tmem] (+)= A[smem] * B[smem]^T, NVFP4 operands with UE4M3 scales in TMEM,
 // 16-element scale blocks.  accumulate == 0 overwrites D.
 __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -349,19 +328,6 @@ __device__ __forceinline__ void scale2(uint32_t x0, uint32_t x1, float s, float 
   asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(s));
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(d));
-}
-
-// 32-byte global load (read-only path) and store; the address is 32-byte
-// aligned.
-__device__ __forceinline__ void ld_nc_v8(const void *p, uint32_t (&r)[8]) {
-  asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "l"(p));
-}
-__device__ __forceinline__ void st_v8(void *p, const uint32_t (&r)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]),
-               "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 
 // e^-64 in binary32 (a normal number).
