@@ -265,79 +265,90 @@ __global__ void __launch_bounds__(kQuantWarps * 32) k_quant(const QuantParams p)
 }
 
 // Requantization of the padded rows of h with the amax the GEMM epilogue
-// reduced (amax reuse): thread per 16-element block, grid-stride over the
-// padded rows [0, padded_offsets[E]) so no lane searches the group offsets.
-// A row whose amax is 0 -- a padding row (the route scan zeroes their amax) or
-// an all-zero row -- gets zero codes, zero scales and S_dec = 1, exactly what
-// quantizing a zero row gives, without reading h.  (r, b) of a lane advance by
-// the fixed stride, so the loop divides once.
-__global__ void __launch_bounds__(256) k_requant_blocks(const QuantParams p, uint32_t nblk) {
+// reduced (amax reuse): thread per two consecutive 16-element blocks of a row
+// (the row's global scales are then computed once for both), grid-stride over
+// the padded rows [0, padded_offsets[E]) so no lane searches the group
+// offsets.  A row whose amax is 0 -- a padding row (the route scan zeroes
+// their amax) or an all-zero row -- gets zero codes, zero scales and S_dec = 1,
+// exactly what quantizing a zero row gives, without reading h.  (r, b2) of a
+// lane advance by the fixed stride, so the loop divides once.  At most 40
+// registers, so that six CTAs (48 warps) stay resident per SM: on the
+// Qwen3-30B-A3B-shaped layer 54 us, against 57 us at 44 registers (five CTAs)
+// and 61 us with one block per thread.
+__global__ void __launch_bounds__(256, 6) k_requant_blocks(const QuantParams p, uint32_t npair) {
   const int lane = threadIdx.x & 31;
   const int64_t K = p.K;
   int64_t rows = __ldg(p.padded_offsets + p.E);
   if (rows > p.rows_cap) rows = p.rows_cap;
   if (rows < 0) rows = 0;
-  const uint32_t total = (uint32_t)rows * nblk;
+  const uint32_t total = (uint32_t)rows * npair;
   const uint32_t stride = gridDim.x * blockDim.x;        // a multiple of 32
-  const uint32_t step_r = stride / nblk, step_b = stride - step_r * nblk;
+  const uint32_t step_r = stride / npair, step_b = stride - step_r * npair;
   uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
-  uint32_t r = i / nblk, b = i - r * nblk;
-  // warp-uniform trip count: the shuffles below need every lane
+  uint32_t r = i / npair, b2 = i - r * npair;
+  // warp-uniform trip count: the shuffle below needs every lane
   for (uint32_t base = i - lane; base < total; base += stride) {
     const bool valid = i < total;
     const float amax = valid ? __ldg(p.amax_src + (p.amax_rows ? r : 0)) : 0.0f;
-    float s_enc = 1.0f, s_dec = 1.0f;
-    uint32_t sfc = 0;
-    uint2 codes = make_uint2(0, 0);
+    float s_dec = 1.0f;
+    uint32_t sf2 = 0;                 // the two blocks' UE4M3 scales, block 2 b2 in the low byte
+    uint4 codes = make_uint4(0, 0, 0, 0);
     if (amax > 0.0f) {
       const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) +
-                                                         (int64_t)r * K) + b * 2;
-      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+                                                         (int64_t)r * K) + b2 * 4;
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
+      float s_enc;
       global_scales(amax, s_enc, s_dec);
-      // block amax on packed BF16 pairs (exact: a max of BF16 values)
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
+      uint32_t cw[4];
 #pragma unroll
-      for (int j = 1; j < 8; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
-      const float bamax = fmaxf(__low2float(m2), __high2float(m2));
-      sfc = cvt_ue4m3(__fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc));
-      if (sfc != 0) {
-        const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
-        float y[8];
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t w[8] = {v[2 * q].x, v[2 * q].y, v[2 * q].z, v[2 * q].w,
+                               v[2 * q + 1].x, v[2 * q + 1].y, v[2 * q + 1].z, v[2 * q + 1].w};
+        // block amax on packed BF16 pairs (exact: a max of BF16 values)
+        __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          y[2 * j] = __fmul_rn(bf16_lo(w[j]), rr);
-          y[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), rr);
+        for (int j = 1; j < 8; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
+        const float bamax = fmaxf(__low2float(m2), __high2float(m2));
+        const uint32_t sfc = cvt_ue4m3(__fmul_rn(__fdiv_rn(bamax, 6.0f), s_enc));
+        cw[2 * q] = cw[2 * q + 1] = 0;
+        if (sfc != 0) {
+          const float rr = __fdiv_rn(s_enc, ue4m3_value(sfc));
+          float y[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            y[2 * j] = __fmul_rn(bf16_lo(w[j]), rr);
+            y[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), rr);
+          }
+          cw[2 * q] = cvt_e2m1x8(y);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            y[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), rr);
+            y[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), rr);
+          }
+          cw[2 * q + 1] = cvt_e2m1x8(y);
         }
-        codes.x = cvt_e2m1x8(y);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          y[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), rr);
-          y[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), rr);
-        }
-        codes.y = cvt_e2m1x8(y);
+        sf2 |= sfc << (8 * q);
       }
+      codes = make_uint4(cw[0], cw[1], cw[2], cw[3]);
     }
-    // four consecutive blocks of one row sit in lanes 4i..4i+3 (rows start at
-    // multiples of nblk, itself a multiple of 4, and the stride and warp
-    // bases are multiples of 32)
-    const int q4 = lane & ~3;
-    const uint32_t s0 = __shfl_sync(0xffffffffu, sfc, q4);
-    const uint32_t s1 = __shfl_sync(0xffffffffu, sfc, q4 + 1);
-    const uint32_t s2 = __shfl_sync(0xffffffffu, sfc, q4 + 2);
-    const uint32_t s3 = __shfl_sync(0xffffffffu, sfc, q4 + 3);
+    // the four blocks 4m..4m+3 of a row sit in lanes 2j, 2j+1: a row's pairs
+    // start at an even index (npair is even) and the stride and the warp
+    // bases are multiples of 32
+    const uint32_t sf_hi = __shfl_down_sync(0xffffffffu, sf2, 1);
     if (valid) {
-      if (b == 0) p.s_dec[r] = s_dec;
-      *reinterpret_cast<uint2 *>(p.q + (int64_t)r * (K >> 1) + (int64_t)b * 8) = codes;
-      if ((lane & 3) == 0)
-        *reinterpret_cast<uint32_t *>(p.sf + sf_offset(p.sf_layout, r, b, K, p.rows_cap)) =
-            s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      if (b2 == 0) p.s_dec[r] = s_dec;
+      *reinterpret_cast<uint4 *>(p.q + (int64_t)r * (K >> 1) + (int64_t)b2 * 16) = codes;
+      if ((lane & 1) == 0)
+        *reinterpret_cast<uint32_t *>(p.sf + sf_offset(p.sf_layout, r, 2 * (int64_t)b2, K, p.rows_cap)) =
+            sf2 | (sf_hi << 16);
     }
     i += stride;
     r += step_r;
-    b += step_b;
-    if (b >= nblk) {
-      b -= nblk;
+    b2 += step_b;
+    if (b2 >= npair) {
+      b2 -= npair;
       ++r;
     }
   }
@@ -393,16 +404,19 @@ cudaError_t launch_quant(const QuantParams &p, cudaStream_t s) {
     // h is requantized with the amax the GEMM epilogue reduced; there is no
     // requantization that computes its own amax
     if (p.compute_row_amax) return cudaErrorInvalidValue;
-    const uint32_t nblk = (uint32_t)(p.K / 16);
-    // every padded row below rows_cap, every block; 32-bit indices
-    if (p.rows_cap * (int64_t)nblk >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-    int64_t blocks = (p.rows_cap * nblk + 255) / 256;
-    // 16 CTAs of 256 threads per SM (two waves of 8): measured 4-5 us faster on
-    // the moe30b layer than one resident wave of 8, and 4 per SM slower
+    // two 16-element blocks per thread; a row holds a multiple of four blocks
+    if (p.K % 64 != 0) return cudaErrorInvalidValue;
+    const uint32_t npair = (uint32_t)(p.K / 32);
+    // every padded row below rows_cap, every pair of blocks; 32-bit indices
+    if (p.rows_cap * (int64_t)npair >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    int64_t blocks = (p.rows_cap * npair + 255) / 256;
+    // 16 CTAs of 256 threads per SM, in waves of the six that fit (with one
+    // block per thread, 16 per SM ran 4-5 us faster on the moe30b layer than
+    // one resident wave of 8, and 4 per SM slower)
     const int64_t persistent = (int64_t)num_sms() * 16;
     if (blocks > persistent) blocks = persistent;
     if (blocks < 1) blocks = 1;
-    k_requant_blocks<<<(unsigned)blocks, 256, 0, s>>>(p, nblk);
+    k_requant_blocks<<<(unsigned)blocks, 256, 0, s>>>(p, npair);
     return cudaGetLastError();
   }
   const int64_t nb = (p.K + 511) / 512;   // 16-element blocks per lane
